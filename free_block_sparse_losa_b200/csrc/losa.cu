@@ -1,0 +1,332 @@
+// C ABI of the LoSA hot path (declared in include/losa.h): host-side argument checks, TMA descriptor encoding and
+// kernel launches. All device work is in the kernels included below; nothing here computes on the host.
+#include "losa.h"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+namespace losa {
+// Per-device error word written by kernels (bitwise OR of the codes below), read and cleared by
+// losa_get_device_error.
+__device__ unsigned int g_device_error = 0;
+constexpr unsigned int kDevErrTimeout = 1u;
+constexpr unsigned int kDevErrBadData = 2u;
+}  // namespace losa
+
+#include "attn_f32.cuh"
+#include "attn_tc.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+using namespace losa;
+
+namespace {
+
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+constexpr int kMaxSelectItems = 32768;   // longest-first order is sorted by one CTA in shared memory
+constexpr int kMaxSelectBlocks = 8192;   // per-row sort in shared memory
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Generic shape consistency (independent of which kernels exist).
+losa_status check_shape(const losa_shape* s) {
+    if (!s) return LOSA_ERR_INVALID_ARG;
+    if (s->heads <= 0 || s->n_tokens <= 0 || s->head_dim <= 0 || s->block_q <= 0 || s->block_k <= 0)
+        return LOSA_ERR_INVALID_ARG;
+    if (s->n_padded < s->n_tokens || s->n_padded % s->block_q != 0 || s->n_padded % s->block_k != 0)
+        return LOSA_ERR_INVALID_ARG;
+    // Every block must hold at least one real token.
+    if (s->n_padded - s->n_tokens >= s->block_q || s->n_padded - s->n_tokens >= s->block_k)
+        return LOSA_ERR_INVALID_ARG;
+    if (s->dtype != LOSA_DTYPE_BF16 && s->dtype != LOSA_DTYPE_F32) return LOSA_ERR_INVALID_ARG;
+    if ((long long)s->heads * s->n_padded * s->head_dim > (1ll << 40)) return LOSA_ERR_INVALID_ARG;
+    return LOSA_OK;
+}
+
+bool tc_shape(const losa_shape* s) {
+    return s->dtype == LOSA_DTYPE_BF16 && s->head_dim == kTcDim && s->block_q == kTcRows && s->block_k == kTcRows &&
+           s->n_padded / kTcRows <= 1024;
+}
+
+bool f32_shape(const losa_shape* s) {
+    return s->dtype == LOSA_DTYPE_F32 && (s->head_dim == 64 || s->head_dim == 128) && s->block_q == s->block_k &&
+           (s->block_q == 32 || s->block_q == 64 || s->block_q == 128);
+}
+
+losa_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LOSA_OK : LOSA_ERR_CUDA;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time dependency on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Tensor map over a [rows][128] bf16 matrix, boxes of 128 rows x 64 columns, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)kTcDim, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)kTcDim * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTcRows};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <TcMode MODE>
+losa_status launch_tc(const losa_shape* s, const void* q, const void* k, const void* v, float scale,
+                      const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
+                      float* mass, cudaStream_t stream) {
+    const uint64_t rows = (uint64_t)s->heads * s->n_padded;
+    CUtensorMap tq, tk, tv;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows)) return LOSA_ERR_CUDA;
+    if (!make_tile_map(&tv, v ? v : k, rows)) return LOSA_ERR_CUDA;
+    TcArgs a;
+    a.H = s->heads;
+    a.N = s->n_tokens;
+    a.Np = s->n_padded;
+    a.nq = s->n_padded / kTcRows;
+    a.nk = s->n_padded / kTcRows;
+    a.n_items = s->heads * a.nq;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.indptr = indptr;
+    a.kv_idx = kv_idx;
+    a.order = order;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.lse = lse;
+    a.mass = mass;
+    a.wait_limit_ns = g_wait_limit_ns;
+    const int sms = sm_count();
+    if (sms <= 0) return LOSA_ERR_CUDA;
+    const int grid = a.n_items < sms ? a.n_items : sms;
+    const uint32_t smem = tc_smem_bytes(MODE);
+    if (cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    attn_tc_kernel<MODE><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
+    return launch_status();
+}
+
+template <int D>
+losa_status launch_f32(const losa_shape* s, const void* q, const void* k, const void* v, float scale,
+                       const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
+                       float* mass, cudaStream_t stream) {
+    F32Args a;
+    a.q = static_cast<const float*>(q);
+    a.k = static_cast<const float*>(k);
+    a.v = static_cast<const float*>(v);
+    a.H = s->heads;
+    a.N = s->n_tokens;
+    a.Np = s->n_padded;
+    a.R = s->block_q;
+    a.C = s->block_k;
+    a.nq = s->n_padded / s->block_q;
+    a.nk = s->n_padded / s->block_k;
+    a.scale = scale;
+    a.indptr = indptr;
+    a.kv_idx = kv_idx;
+    a.order = order;
+    a.o = static_cast<float*>(o);
+    a.lse = lse;
+    const int items = a.H * a.nq;
+    const size_t smem_fwd = (size_t)2 * a.C * D * sizeof(float);
+    if (cudaFuncSetAttribute(attn_f32_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_fwd) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    attn_f32_fwd_kernel<D><<<items, a.R, smem_fwd, stream>>>(a);
+    losa_status st = launch_status();
+    if (st != LOSA_OK || !mass) return st;
+    const size_t smem_mass = (size_t)a.C * D * sizeof(float) + (size_t)a.R * sizeof(float);
+    if (cudaFuncSetAttribute(mass_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_mass) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    a.indptr = nullptr;
+    a.order = nullptr;
+    mass_f32_kernel<D><<<items, a.R, smem_mass, stream>>>(a, mass);
+    return launch_status();
+}
+
+int next_pow2(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+size_t select_ws_bytes(const losa_shape* s) {
+    const size_t rows = (size_t)s->heads * (s->n_padded / s->block_q);
+    const size_t nk = (size_t)(s->n_padded / s->block_k);
+    const size_t staged = (rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
+    const size_t counts = (rows * sizeof(int32_t) + 255) & ~(size_t)255;
+    return staged + counts;
+}
+
+}  // namespace
+
+extern "C" {
+
+int losa_version(void) { return 100; }
+
+const char* losa_status_string(losa_status st) {
+    switch (st) {
+        case LOSA_OK: return "LOSA_OK";
+        case LOSA_ERR_INVALID_ARG: return "LOSA_ERR_INVALID_ARG";
+        case LOSA_ERR_UNSUPPORTED: return "LOSA_ERR_UNSUPPORTED";
+        case LOSA_ERR_CAPACITY: return "LOSA_ERR_CAPACITY";
+        case LOSA_ERR_CUDA: return "LOSA_ERR_CUDA";
+        case LOSA_ERR_DEVICE_FAULT: return "LOSA_ERR_DEVICE_FAULT";
+        case LOSA_ERR_TIMEOUT: return "LOSA_ERR_TIMEOUT";
+    }
+    return "LOSA_ERR_UNKNOWN";
+}
+
+void losa_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns = limit_ns < 1000 ? 1000 : limit_ns; }
+
+losa_status losa_dense_profile(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                               void* o, float* lse, float* mass, cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LOSA_ERR_INVALID_ARG;
+    if (mass && !aligned16(lse)) return LOSA_ERR_INVALID_ARG;
+    if (lse && !aligned16(lse)) return LOSA_ERR_INVALID_ARG;
+    if (mass && !aligned16(mass)) return LOSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
+    if (tc_shape(shape)) {
+        st = launch_tc<TcMode::Fwd>(shape, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, nullptr, stream);
+        if (st != LOSA_OK || !mass) return st;
+        return launch_tc<TcMode::Mass>(shape, q, k, nullptr, scale, nullptr, nullptr, nullptr, nullptr, lse, mass,
+                                       stream);
+    }
+    if (f32_shape(shape)) {
+        if (shape->head_dim == 64)
+            return launch_f32<64>(shape, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, mass, stream);
+        return launch_f32<128>(shape, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, mass, stream);
+    }
+    return LOSA_ERR_UNSUPPORTED;
+}
+
+size_t losa_select_workspace_bytes(const losa_shape* shape) {
+    if (check_shape(shape) != LOSA_OK) return 0;
+    return select_ws_bytes(shape);
+}
+
+losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
+                        int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
+                        size_t ws_bytes, cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_INVALID_ARG;
+    if (!aligned16(mass) || !indptr || !kv_block_idx || !order || !aligned16(workspace)) return LOSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
+         reinterpret_cast<uintptr_t>(order)) & 3u)
+        return LOSA_ERR_INVALID_ARG;
+    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
+    const long long rows = (long long)shape->heads * nq;
+    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
+    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
+    if (ws_bytes < select_ws_bytes(shape)) return LOSA_ERR_CAPACITY;
+
+    int32_t* staged = static_cast<int32_t*>(workspace);
+    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
+    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
+
+    const int n2 = next_pow2(nk);
+    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
+    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem1) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, counts,
+                                                                                         staged);
+    if ((st = launch_status()) != LOSA_OK) return st;
+
+    const int r2 = next_pow2((int)rows);
+    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
+    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem2) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
+    if ((st = launch_status()) != LOSA_OK) return st;
+
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
+    return launch_status();
+}
+
+losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                             const int32_t* indptr, const int32_t* kv_block_idx, const int32_t* order, void* o,
+                             float* lse, cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !indptr || !kv_block_idx)
+        return LOSA_ERR_INVALID_ARG;
+    if (lse && !aligned16(lse)) return LOSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
+    if (tc_shape(shape))
+        return launch_tc<TcMode::Fwd>(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
+    if (f32_shape(shape)) {
+        if (shape->head_dim == 64)
+            return launch_f32<64>(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
+        return launch_f32<128>(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
+    }
+    return LOSA_ERR_UNSUPPORTED;
+}
+
+losa_status losa_get_device_error(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LOSA_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess) return LOSA_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (word && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return LOSA_ERR_CUDA;
+    if (word & kDevErrTimeout) return LOSA_ERR_TIMEOUT;
+    if (word & kDevErrBadData) return LOSA_ERR_DEVICE_FAULT;
+    return LOSA_OK;
+}
+
+}  // extern "C"
+
+// Bounded-wait self-test: one thread waits on a barrier whose single expected arrival never happens.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t addr = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(addr, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wait_bounded(addr, 0, limit_ns);
+    __syncthreads();
+}
+
+extern "C" losa_status losa_selftest_wait_timeout(uint32_t limit_ns, cudaStream_t stream) {
+    selftest_wait_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns);
+    return launch_status();
+}

@@ -1,0 +1,74 @@
+"""Device-buffer harness around the C ABI: allocates the caller-owned buffers of one attention layer with
+PyTorch (device memory and streams only) and calls the three entry points in order. No computation happens
+here; every step runs in the library's kernels."""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import (DTYPE_BF16, DTYPE_F32, losa_dense_profile, losa_select, losa_select_workspace_bytes,
+               losa_sparse_attn, make_shape)
+
+
+def host_tokens_to_device(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    """[H][Np][d] host tokens (fp32 values, or uint16 bf16 bit patterns) -> contiguous device tensor."""
+    if dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(device)
+
+
+def device_tokens_to_f32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()
+
+
+@dataclass
+class LayerBuffers:
+    heads: int
+    n_tokens: int
+    n_padded: int
+    head_dim: int
+    block: int
+    dtype: str
+    device: str = "cuda"
+
+    def __post_init__(self):
+        self.shape = make_shape(self.heads, self.n_tokens, self.n_padded, self.head_dim, self.block, self.block,
+                                self.dtype)
+        self.nq = self.n_padded // self.block
+        self.nk = self.nq
+        self.rows = self.heads * self.nq
+        tdt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        dev = self.device
+        self.o = torch.empty((self.heads, self.n_padded, self.head_dim), dtype=tdt, device=dev)
+        self.lse = torch.empty((self.heads, self.n_padded), dtype=torch.float32, device=dev)
+        self.mass = torch.empty((self.heads, self.nq, self.nk), dtype=torch.float32, device=dev)
+        self.indptr = torch.empty(self.rows + 1, dtype=torch.int32, device=dev)
+        self.kv_idx = torch.empty(self.rows * self.nk, dtype=torch.int32, device=dev)
+        self.order = torch.empty(self.rows, dtype=torch.int32, device=dev)
+        ws = losa_select_workspace_bytes(self.shape)
+        self.workspace = torch.empty((ws + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+
+    @classmethod
+    def for_config(cls, cfg, device="cuda"):
+        return cls(cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block, cfg.dtype, device)
+
+    def profile(self, q, k, v, scale, with_mass=True, stream=None):
+        losa_dense_profile(self.shape, q, k, v, scale, self.o, self.lse, self.mass if with_mass else None,
+                           stream=stream)
+
+    def select(self, tau, mass=None, stream=None):
+        losa_select(self.shape, self.mass if mass is None else mass, tau, self.indptr, self.kv_idx, self.order,
+                    self.workspace, stream=stream)
+
+    def sparse(self, q, k, v, scale, out=None, lse=None, stream=None, order=True):
+        losa_sparse_attn(self.shape, q, k, v, scale, self.indptr, self.kv_idx, self.order if order else None,
+                         self.o if out is None else out, lse, stream=stream)
+
+    def csr_host(self):
+        indptr = self.indptr.cpu().numpy()
+        nnz = int(indptr[-1])
+        return indptr, self.kv_idx[:nnz].cpu().numpy(), self.order.cpu().numpy()

@@ -1,0 +1,146 @@
+/*
+ * losa.h — C ABI of the LoSA hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method is the one of the page "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion
+ * Acceleration": at one dense denoising step, measure the exact attention mass of every (head, query block,
+ * key block); for each head and query block keep the smallest set of key blocks whose mass reaches a
+ * threshold tau; at every later step run block-sparse attention over those frozen blocks only.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is DEVICE memory owned by the caller (allocated on the current device). The
+ *     library allocates nothing and keeps no state between calls other than one per-device error word.
+ *   - Every call is asynchronous and stream-ordered on `stream`, except losa_get_device_error (which
+ *     synchronises the stream). Host-side argument checks run first and return before anything is launched.
+ *   - Token tensors q, k, v, o are [H][Np][d] row-major, d contiguous: head h, token t starts at element
+ *     (h * Np + t) * d. Tokens are the video latent's (t, y, x) grid flattened row-major, padded from N to Np
+ *     (a multiple of the block sizes, N <= Np < N + block). Keys t >= N take no part in any softmax; output
+ *     rows t >= N are written but carry no meaning. Base pointers must be 16-byte aligned.
+ *   - An "item" is one (head, query block) pair with id h * nq + i, nq = Np / block_q, nk = Np / block_k.
+ *   - Status codes below; LOSA_ERR_CUDA covers launch failures reported by the CUDA runtime.
+ *
+ * Supported shapes: dtype BF16 with head_dim 128 and block_q = block_k = 128 (tensor-core path), or dtype F32
+ * with head_dim 64 or 128 and block_q = block_k in {32, 64, 128} (exact fp32 path for small checks).
+ */
+#ifndef LOSA_H
+#define LOSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LOSA_OK = 0,
+    LOSA_ERR_INVALID_ARG = -1,   /* null / misaligned pointer, inconsistent shape, tau outside (0, 1]      */
+    LOSA_ERR_UNSUPPORTED = -2,   /* a valid shape this build has no kernel for                          */
+    LOSA_ERR_CAPACITY = -3,      /* an output or workspace buffer is smaller than the worst case          */
+    LOSA_ERR_CUDA = -4,          /* the CUDA runtime reported an error at launch or synchronisation      */
+    LOSA_ERR_DEVICE_FAULT = -5,  /* a kernel detected invalid data (bad block index, non-finite mass)   */
+    LOSA_ERR_TIMEOUT = -6        /* a kernel's bounded wait ran out; the kernel exited cleanly           */
+} losa_status;
+
+enum { LOSA_DTYPE_F32 = 0, LOSA_DTYPE_BF16 = 1 };
+
+typedef struct {
+    int32_t heads;     /* H                                                        */
+    int32_t n_tokens;  /* N, real tokens                                            */
+    int32_t n_padded;  /* Np, multiple of block_q and block_k, N <= Np < N + block  */
+    int32_t head_dim;  /* d                                                        */
+    int32_t block_q;   /* R, query block size                                       */
+    int32_t block_k;   /* C, key/value block size                                   */
+    int32_t dtype;     /* LOSA_DTYPE_BF16 or LOSA_DTYPE_F32, for q, k, v and o      */
+} losa_shape;
+
+/*
+ * Dense profiling step (LoSA page, Motivation Summary: A = softmax(Q K^T / sqrt(d)) and the block attention
+ * mass M(i, j) = sum over q in query block i and k in key block j of A(q, k); Methodology Summary: the masses are
+ * exact because construction coincides with a dense step).
+ *   q, k, v  : [H][Np][d] input tokens (dtype of the shape).
+ *   scale    : logit scale, normally 1 / sqrt(d).
+ *   o        : [H][Np][d] output, dense softmax attention (same dtype).
+ *   lse      : [H][Np] fp32, natural log of each row's softmax denominator, ln sum_k exp(scale q.k).
+ *              May be NULL only when mass is NULL.
+ *   mass     : [H][nq][nk] fp32 or NULL. Row (h, i) is M(i, .) divided by R_i, the real rows of query block i,
+ *              so every row sums to one. NULL runs the forward pass only (an ordinary dense step).
+ * With mass != NULL a second pass recomputes Q K^T tile by tile and sums exp(s - lse) into block sums without
+ * materialising the probability matrix.
+ */
+losa_status losa_dense_profile(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                               void* o, float* lse, float* mass, cudaStream_t stream);
+
+/*
+ * Mass-threshold selection (LoSA page, Methodology Summary, "One-time pattern construction": sort the key
+ * blocks of one (head, query block) by decreasing mass and keep the shortest prefix whose mass reaches
+ * theta times the block's total).
+ *   mass          : [H][nq][nk] fp32, non-negative, finite (as written by losa_dense_profile).
+ *   tau           : retained-mass threshold in (0, 1].
+ *   indptr        : [H*nq + 1] int32 output; row r's kept blocks are kv_block_idx[indptr[r] .. indptr[r+1]).
+ *                   indptr[H*nq] = nnz stays on the device; reading it back is the caller's choice.
+ *   kv_block_idx  : [idx_capacity] int32 output, kept key-block indices of each row in ascending order.
+ *   idx_capacity  : must be >= H*nq*nk (the worst case), else LOSA_ERR_CAPACITY.
+ *   order         : [H*nq] int32 output, item ids by list length descending, ties by ascending id (the
+ *                   longest-first work order losa_sparse_attn consumes). At most 32768 items per call.
+ *   workspace     : device scratch of at least losa_select_workspace_bytes(shape) bytes (16-byte aligned);
+ *                   its contents on entry do not matter.
+ * Rule per row: order blocks by (mass descending, index ascending); u_j = ceil(M_j * 2^52) as 64-bit integers;
+ * T = ceil(tau * sum_j u_j) in IEEE double; keep the first s >= 1 blocks whose integer prefix reaches T. The
+ * integer prefix makes the result independent of summation order, and tau = 1 keeps exactly the non-zero blocks.
+ * A negative or non-finite mass sets the device error word (LOSA_ERR_DEVICE_FAULT) and is treated as zero.
+ */
+losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
+                        int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of device workspace losa_select needs for this shape (0 if the shape is invalid). */
+size_t losa_select_workspace_bytes(const losa_shape* shape);
+
+/*
+ * Block-sparse attention over a frozen pattern (LoSA page, Methodology Summary, "Sparse attention with a frozen
+ * pattern": each query attends only to the keys of its retained blocks, and the softmax denominator runs over
+ * those keys only).
+ *   q, k, v       : [H][Np][d] tokens of the current step (they may differ from the profiled step's).
+ *   indptr, kv_block_idx : the CSR lists written by losa_select (any order within a row is accepted; every
+ *                   index must lie in [0, nk), every row must be non-empty).
+ *   order         : [H*nq] permutation of item ids giving the work order (longest list first for balance),
+ *                   or NULL for ascending item order.
+ *   o             : [H][Np][d] output; lse: [H][Np] fp32 output or NULL.
+ * An out-of-range block index or an empty row sets the device error word (LOSA_ERR_DEVICE_FAULT); the
+ * affected rows are left unspecified.
+ */
+losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                             const int32_t* indptr, const int32_t* kv_block_idx, const int32_t* order, void* o,
+                             float* lse, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error word: LOSA_OK,
+ * LOSA_ERR_DEVICE_FAULT, LOSA_ERR_TIMEOUT, or LOSA_ERR_CUDA if the synchronisation itself failed.
+ */
+losa_status losa_get_device_error(cudaStream_t stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on a shared-memory barrier nothing ever
+ * completes, for at most `limit_ns` nanoseconds, then records LOSA_ERR_TIMEOUT in the device error word and
+ * exits. No GPU fault is involved; read the result with losa_get_device_error.
+ */
+losa_status losa_selftest_wait_timeout(uint32_t limit_ns, cudaStream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, of every wait inside the library's kernels on this process (default 2e9).
+ * Exposed for tests; values below 1000 are raised to 1000.
+ */
+void losa_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Human-readable name of a status code (static string). */
+const char* losa_status_string(losa_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int losa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOSA_H */

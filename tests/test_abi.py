@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point include/losa.h declares, and its
+host-side argument checks reject bad calls before anything is launched (no GPU needed: none of these calls
+reaches the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_block_sparse_losa_b200 as L
+from free_block_sparse_losa_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(losa_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert {"losa_dense_profile", "losa_select", "losa_sparse_attn", "losa_select_workspace_bytes",
+            "losa_get_device_error", "losa_status_string"} <= names
+    raw = ctypes.CDLL(L.library_path())
+    for n in sorted(names):
+        assert hasattr(raw, n), n
+
+
+def test_status_strings(lib):
+    for code, name in L.STATUS.items():
+        assert L.losa_status_string(code) == name
+    assert L.losa_version() >= 100
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails its host checks first
+
+
+def test_shape_validation(lib):
+    good = L.make_shape(2, 1000, 1024, 128, 128, 128, "bf16")
+    assert L.losa_select_workspace_bytes(good) > 0
+    bad = [
+        L.make_shape(0, 1000, 1024, 128, 128, 128, "bf16"),      # no heads
+        L.make_shape(2, 1100, 1024, 128, 128, 128, "bf16"),      # N > Np
+        L.make_shape(2, 1000, 1000, 128, 128, 128, "bf16"),      # Np not a multiple of the block
+        L.make_shape(2, 800, 1024, 128, 128, 128, "bf16"),       # an all-padding block
+        L.make_shape(2, 1000, 1024, 128, 128, 128, 7),           # unknown dtype
+    ]
+    for s in bad:
+        assert L.losa_select_workspace_bytes(s) == 0
+        assert L.losa_dense_profile(s, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, stream=0,
+                                    raise_on_error=False) == -1
+        assert L.losa_sparse_attn(s, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, None, FAKE, stream=0,
+                                  raise_on_error=False) == -1
+    assert lib.losa_dense_profile(None, None, None, None, 0.1, None, None, None, None) == -1
+
+
+def test_pointer_and_tau_validation(lib):
+    s = L.make_shape(2, 1000, 1024, 128, 128, 128, "bf16")
+    # misaligned / null pointers
+    assert L.losa_dense_profile(s, FAKE + 2, FAKE, FAKE, 0.1, FAKE, FAKE, None, stream=0, raise_on_error=False) == -1
+    assert L.losa_dense_profile(s, FAKE, FAKE, None, 0.1, FAKE, FAKE, None, stream=0, raise_on_error=False) == -1
+    # mass requested without lse
+    assert L.losa_dense_profile(s, FAKE, FAKE, FAKE, 0.1, FAKE, None, FAKE, stream=0, raise_on_error=False) == -1
+    assert L.losa_dense_profile(s, FAKE, FAKE, FAKE, float("nan"), FAKE, FAKE, None, stream=0,
+                                raise_on_error=False) == -1
+    ws = L.losa_select_workspace_bytes(s)
+    for tau in (0.0, -1.0, 1.5, float("nan")):
+        assert L.losa_select(s, FAKE, tau, FAKE, FAKE, FAKE, FAKE, idx_capacity=2 * 8 * 8, ws_bytes=ws, stream=0,
+                             raise_on_error=False) == -1
+
+
+def test_capacity_and_unsupported(lib):
+    s = L.make_shape(2, 1000, 1024, 128, 128, 128, "bf16")
+    ws = L.losa_select_workspace_bytes(s)
+    rows, nk = 2 * 8, 8
+    assert L.losa_select(s, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=rows * nk - 1, ws_bytes=ws, stream=0,
+                         raise_on_error=False) == -3
+    assert L.losa_select(s, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=rows * nk, ws_bytes=ws - 1, stream=0,
+                         raise_on_error=False) == -3
+    # bf16 is implemented for head_dim 128 with 128-blocks only
+    s64 = L.make_shape(2, 1000, 1024, 64, 128, 128, "bf16")
+    assert L.losa_dense_profile(s64, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, None, stream=0, raise_on_error=False) == -2
+    # more items than one selection call orders
+    big = L.make_shape(300, 130000, 130048, 128, 128, 128, "bf16")
+    wsb = L.losa_select_workspace_bytes(big)
+    assert L.losa_select(big, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40, ws_bytes=wsb, stream=0,
+                         raise_on_error=False) == -2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setenv("LOSA_LIBRARY", "/nonexistent/liblosa.so")
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(RuntimeError):
+        L.load()

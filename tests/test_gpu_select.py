@@ -1,0 +1,91 @@
+"""GPU parity of losa_select against the oracle fed the same fp32 masses: CSR lists and the longest-first
+work order must match bit for bit (LoSA page, Methodology Summary, "One-time pattern construction")."""
+import numpy as np
+import pytest
+import torch
+
+import free_block_sparse_losa_b200 as L
+from tests.gpu_util import compare_select, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _masses(rng, rows, nk, kind):
+    if kind == "exp":
+        m = rng.exponential(size=(rows, nk)) ** 4
+    elif kind == "ties":
+        m = rng.integers(0, 5, size=(rows, nk)).astype(np.float64)
+        m[:, 0] += 1.0
+    elif kind == "peaked":  # few dominant blocks, long tail spanning many decades (like real attention)
+        m = np.exp(rng.standard_normal((rows, nk)) * 8.0)
+    elif kind == "uniform":
+        m = np.ones((rows, nk))
+    m = m / m.sum(axis=1, keepdims=True)
+    return m.astype(np.float32)
+
+
+def _run(shape_args, m, tau, oracle):
+    H, nq, nk, R, C = shape_args
+    Np = nk * C
+    shape = L.make_shape(H, Np - 1, Np, 128, R, C, "bf16")
+    dev = torch.from_numpy(m.reshape(H * nq * nk)).cuda()
+    rows = H * nq
+    indptr = torch.full((rows + 1,), -7, dtype=torch.int32, device="cuda")
+    idx = torch.full((rows * nk,), -7, dtype=torch.int32, device="cuda")
+    order = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(L.losa_select_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    L.losa_select(shape, dev, tau, indptr, idx, order, ws)
+    assert L.losa_get_device_error() == 0
+    gi = indptr.cpu().numpy()
+    nnz = int(gi[-1])
+    gk = idx.cpu().numpy()
+    # nothing written past nnz
+    assert (gk[nnz:] == -7).all()
+    return compare_select(gi, gk[:nnz], order.cpu().numpy(), m.reshape(rows, nk), tau, oracle)
+
+
+@pytest.mark.parametrize("H,nb", [(1, 1), (1, 2), (3, 4), (2, 31), (2, 64), (4, 256), (1, 929), (2, 1024)])
+@pytest.mark.parametrize("kind", ["exp", "ties", "peaked", "uniform"])
+def test_select_matches_oracle(H, nb, kind, oracle_mod):
+    rng = np.random.default_rng(H * 1000 + nb)
+    m = _masses(rng, H * nb, nb, kind)
+    for tau in (0.5, 0.9, 0.99, 1.0):
+        counts = _run((H, nb, nb, 128, 128), m, tau, oracle_mod)
+        assert counts.min() >= 1
+
+
+def test_select_uneven_blocks(oracle_mod):
+    """R = 64, C = 32: more key blocks than query blocks per row."""
+    rng = np.random.default_rng(3)
+    H, nq, nk = 3, 20, 40
+    m = _masses(rng, H * nq, nk, "peaked")
+    for tau in (0.9, 0.99):
+        _run((H, nq, nk, 64, 32), m, tau, oracle_mod)
+
+
+def test_select_full_size_hunyuan_rows(oracle_mod):
+    """22296 rows x 929 blocks (the HunyuanVideo-720p-shaped layer), peaked masses."""
+    rng = np.random.default_rng(4)
+    H, nb = 24, 929
+    m = _masses(rng, H * nb, nb, "peaked")
+    _run((H, nb, nb, 128, 128), m, 0.99, oracle_mod)
+
+
+def test_select_reports_bad_mass():
+    shape = L.make_shape(1, 1023, 1024, 128, 128, 128, "bf16")
+    rows, nk = 8, 8
+    mm = np.full((rows, nk), 1.0 / 8, np.float32)
+    mm[5, 2] = np.nan
+    dev = torch.from_numpy(mm.ravel()).cuda()
+    indptr = torch.empty(rows + 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(rows * nk, dtype=torch.int32, device="cuda")
+    order = torch.empty(rows, dtype=torch.int32, device="cuda")
+    ws = torch.empty(L.losa_select_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    L.losa_select(shape, dev, 0.9, indptr, idx, order, ws)
+    assert L.losa_get_device_error() == -5
+    assert L.losa_get_device_error() == 0  # cleared by the read
