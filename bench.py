@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the LoSA hot path on B200.
+
+One step = the whole hot path over one synthetic attention layer: losa_dense_profile (dense forward + exact block
+masses), losa_select (tau = 0.99 by default) and losa_sparse_attn over the frozen lists. The default workload is the
+HunyuanVideo-720p-shaped layer (24 heads, 33x45x80 token grid, N = 118800 padded to 118912, head_dim 128, bf16,
+128 x 128 blocks), the layer the sparse-attention throughput target is quoted on.
+
+Prints ONE JSON line (rank 0). `value` is the dense-equivalent throughput of losa_sparse_attn, 4*H*N^2*d / t_sparse,
+summed over ranks (weak scaling: every rank runs its own layer); the per-kernel times, the profile+select time, the
+block density, the roofline of each kernel and the oracle's CPU baseline are extra keys.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from losa_synth import CONFIGS, make_layer, sample_items  # noqa: E402
+
+WORKLOADS = {"hunyuan720": 3, "wan14b720": 2, "wan1.3b480": 1, "tiny": 0}
+METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select ms"
+KERNELS_PER_STEP = {"dense_profile": 2, "select": 3, "sparse_attn": 1}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "sm_max_mhz": p.get("sm_max_mhz", 1965.0),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+def work_model(cfg, nnz):
+    """Algorithmic work per call. Tensor FLOPs count 2 per multiply-add; the dense-equivalent figure uses the
+    real token count N, kept-block figures count whole 128 x 128 tiles."""
+    H, N, Np, d, B = cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block
+    nq = Np // B
+    return {
+        "dense_equiv_flop": 4.0 * H * N * N * d,
+        "profile_flop": 6.0 * H * N * N * d,          # Q K^T + P V forward, then Q K^T again for the masses
+        "profile_exp": 2.0 * H * N * N,
+        "sparse_flop": 4.0 * B * B * d * nnz,         # kept tiles only
+        "sparse_exp": float(B * B * nnz),
+        "select_bytes": 4.0 * H * nq * nq + 4.0 * (nnz + 2 * H * nq + 1),  # read M, write CSR + order
+    }
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def roofline(name, bound, work, seconds, pk, unit, traffic=None, peak_kind="sustained"):
+    if bound == "tensor":
+        peak = pk["bf16_tflops_sustained"] if peak_kind == "sustained" else pk["bf16_tflops"]
+        achieved = work / seconds / 1e12
+    elif bound == "hbm":
+        peak = pk["hbm_gbs"]
+        achieved = work / seconds / 1e9
+    else:  # alu (exp unit): 148 SMs x 16 ex2 per clock at the max SM clock
+        peak = 148 * 16 * pk["sm_max_mhz"] * 1e6 / 1e12
+        achieved = work / seconds / 1e12
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": f"{pk['source']} {peak_kind}"
+            if bound == "tensor" else pk["source"]}
+
+
+# ------------------------------------------------------------------------------------------------ CPU oracle
+
+def oracle_inputs(layer):
+    return layer.all_f32("q"), layer.all_f32("k"), layer.all_f32("v")
+
+
+def oracle_threads():
+    import oracle
+    return oracle.num_threads()
+
+
+def oracle_sample_run(cfg, qkv, tau, n_items, seed=7):
+    """The oracle, as it stands, on a seeded sample of (head, query block) items of the workload: dense forward,
+    masses, selection and restricted attention. Returns per-item seconds of each stage."""
+    import oracle
+    q, k, v = qkv
+    items = sample_items(cfg, n_items, seed=seed)[:n_items]
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    R, N = cfg.block, cfg.n_tokens
+    t0 = time.perf_counter()
+    oracle.dense(q, k, v, N, R, scale, items)
+    t1 = time.perf_counter()
+    m = oracle.mass(q, k, N, R, R, scale, items)
+    t2 = time.perf_counter()
+    counts, idx = oracle.select(m.astype(np.float32), tau)
+    t3 = time.perf_counter()
+    # CSR over the sampled items only: rows outside the sample are empty
+    rows = cfg.heads * cfg.n_blocks
+    full_counts = np.zeros(rows, np.int32)
+    full_counts[items] = counts
+    indptr = np.zeros(rows + 1, np.int32)
+    indptr[1:] = np.cumsum(full_counts)
+    kv = np.concatenate([idx[t, :counts[t]] for t in range(len(items))]).astype(np.int32)
+    t4 = time.perf_counter()
+    oracle.sparse(q, k, v, N, R, R, scale, indptr, kv, items)
+    t5 = time.perf_counter()
+    n = len(items)
+    return {"items": n, "dense_s": (t1 - t0) / n, "mass_s": (t2 - t1) / n, "select_s": (t3 - t2) / n,
+            "sparse_s": (t5 - t4) / n, "density": float(counts.sum()) / (n * cfg.n_blocks),
+            "threads": oracle.num_threads()}
+
+
+def cpu_line(cfg, per_item, sample_desc):
+    rows = cfg.heads * cfg.n_blocks
+    work = work_model(cfg, 0)
+    t_sparse = per_item["sparse_s"] * rows
+    return {"value": round(work["dense_equiv_flop"] / t_sparse / 1e12, 6),
+            "unit": "TFLOP/s (dense-equivalent, sparse attention)", "cores": per_item["threads"], "kind": "oracle",
+            "sample": sample_desc, "sparse_attn_ms_extrapolated": round(t_sparse * 1e3, 1),
+            "profile_select_ms_extrapolated": round((per_item["dense_s"] + per_item["mass_s"] +
+                                                     per_item["select_s"]) * rows * 1e3, 1)}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    layer = make_layer(cfg)
+    qkv = oracle_inputs(layer)
+    n_items = args.ref_items or max(1, oracle_threads() // 2)
+    desc = (f"{n_items} seeded (head, query-block) items of {cfg.name} per step (dense forward, masses, "
+            f"selection, restricted attention), fp64 oracle, extrapolated linearly to all "
+            f"{cfg.heads * cfg.n_blocks} items")
+    for _ in range(args.warmup):
+        oracle_sample_run(cfg, qkv, args.tau, max(1, n_items // 4), seed=99)
+    runs = [oracle_sample_run(cfg, qkv, args.tau, n_items, seed=1000 + s) for s in range(args.steps)]
+    per = {k: float(np.mean([r[k] for r in runs])) for k in ("dense_s", "mass_s", "select_s", "sparse_s",
+                                                             "density")}
+    per["threads"] = runs[0]["threads"]
+    c = cpu_line(cfg, per, desc)
+    rows = cfg.heads * cfg.n_blocks
+    step_ms = (per["dense_s"] + per["mass_s"] + per["select_s"] + per["sparse_s"]) * rows * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": c["value"], "unit": c["unit"], "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens,
+                       "head_dim": cfg.head_dim, "block": cfg.block, "tau": args.tau},
+            "sparse_attn_ms": c["sparse_attn_ms_extrapolated"],
+            "profile_select_ms": c["profile_select_ms_extrapolated"],
+            "cpu_baseline": {"value": c["value"], "unit": c["unit"], "cores": c["cores"], "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": c["value"], "unit": c["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------- native path
+
+def run_native(args, cfg):
+    import torch
+    import free_block_sparse_losa_b200 as L
+    from free_block_sparse_losa_b200.harness import LayerBuffers, host_tokens_to_device
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    L.load()
+    layer = make_layer(cfg)
+    q, k, v = (host_tokens_to_device(getattr(layer, n), cfg.dtype) for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    buf = LayerBuffers.for_config(cfg)
+    stream = torch.cuda.current_stream()
+
+    def step(ev):
+        ev[0].record(stream)
+        buf.profile(q, k, v, scale)
+        ev[1].record(stream)
+        buf.select(args.tau)
+        ev[2].record(stream)
+        buf.sparse(q, k, v, scale)
+        ev[3].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
+    for _ in range(args.warmup):
+        step(mk())
+    torch.cuda.synchronize()
+    if L.losa_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    nnz = int(buf.indptr[-1].item())
+
+    evs = [mk() for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for e in evs:
+            step(e)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    prof_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    sel_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    spa_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    t_sparse = max_over_ranks(sum(spa_ms) / 1e3)
+    t_prof = max_over_ranks(sum(prof_ms) / 1e3)
+    t_sel = max_over_ranks(sum(sel_ms) / 1e3)
+    status = L.losa_get_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error in timed region: {status}")
+
+    work = work_model(cfg, nnz)
+    K = args.steps
+    value = world * K * work["dense_equiv_flop"] / t_sparse / 1e12
+
+    # end to end through the C ABI with host buffers: pinned Q/K/V -> device, sparse attention, O -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(buf.o.shape, dtype=buf.o.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            buf.sparse(dq, dk, dv, scale)
+            ho.copy_(buf.o, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+        if L.losa_get_device_error() != 0:
+            raise RuntimeError("device error in the end-to-end loop")
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+        d2h = ho.numel() * ho.element_size()
+        e2e = {"value": round(world * K * work["dense_equiv_flop"] / t_e2e / 1e12, 3),
+               "unit": "TFLOP/s (dense-equivalent, sparse attention incl. host copies)",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_call": round(t_e2e / K * 1e3, 3)}
+
+    pk = peaks()
+    per_sparse = t_sparse / K
+    per_prof = t_prof / K
+    per_sel = t_sel / K
+    roof = {
+        "dense_profile": roofline("attn_tc_kernel<Fwd> + attn_tc_kernel<Mass> (losa_dense_profile)", "tensor",
+                                  work["profile_flop"], per_prof, pk, "TFLOP/s"),
+        "select": roofline("select_rows + select_finalize + select_scatter (losa_select)", "hbm",
+                           work["select_bytes"], per_sel, pk, "GB/s"),
+        "sparse_attn": roofline("attn_tc_kernel<Fwd> over retained lists (losa_sparse_attn)", "tensor",
+                                work["sparse_flop"], per_sparse, pk, "TFLOP/s"),
+    }
+    dominant = max(("dense_profile", per_prof), ("select", per_sel), ("sparse_attn", per_sparse),
+                   key=lambda x: x[1])[0]
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s (dense-equivalent, sparse attention)",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic (seeded grid-structured Q/K/V, see DESIGN.md)",
+        "config": {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens, "n_padded": cfg.n_padded,
+                   "head_dim": cfg.head_dim, "block": cfg.block, "tau": args.tau,
+                   "l2": "inputs larger than L2 (3 x %.0f MB of Q/K/V per layer)" % (q.numel() * 2 / 1e6),
+                   "parallelism": f"replicas x{world} (one independent layer per GPU)"},
+        "sparse_attn_ms": round(per_sparse * 1e3, 3),
+        "profile_ms": round(per_prof * 1e3, 3),
+        "select_ms": round(per_sel * 1e3, 3),
+        "profile_select_ms": round((per_prof + per_sel) * 1e3, 3),
+        "dense_equiv_tflops": round(K * work["dense_equiv_flop"] / t_sparse / 1e12, 3),
+        "kept_block_tflops": round(work["sparse_flop"] / per_sparse / 1e12, 3),
+        "block_density": round(nnz / (cfg.heads * cfg.n_blocks ** 2), 5),
+        "nnz_blocks": nnz,
+        "roofline": roof[dominant],
+        "rooflines": roof,
+        "gpu_launches": K * sum(KERNELS_PER_STEP.values()),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_cpu = args.cpu_items or oracle_threads()
+        per = oracle_sample_run(cfg, oracle_inputs(layer), args.tau, n_cpu)
+        line["cpu_baseline"] = cpu_line(cfg, per, f"{n_cpu} seeded items of {cfg.name} (dense forward, "
+                                        f"masses, selection, restricted attention), extrapolated to all "
+                                        f"{cfg.heads * cfg.n_blocks} items")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="hunyuan720")
+    ap.add_argument("--tau", type=float, default=0.99)
+    ap.add_argument("--cpu-items", type=int, default=0, help="oracle sample size (0: one item per host thread)")
+    ap.add_argument("--ref-items", type=int, default=0, help="reference-arm items per step (0: half the threads)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    cfg = CONFIGS[WORKLOADS[args.workload]]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_native(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
