@@ -330,3 +330,83 @@ extern "C" losa_status losa_selftest_wait_timeout(uint32_t limit_ns, cudaStream_
     selftest_wait_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns);
     return launch_status();
 }
+
+// ------------------------------------------------------------------------------------------------------------------
+// Selection without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at call time: a serving process that reserved nearly all of the GPU's
+// memory for its own pool at start-up (a cudaMalloc then fails or would bypass its accounting), a plugin whose host
+// framework owns every buffer and offers no workspace, or a latency-critical path where cudaMalloc / cudaFree may
+// synchronise the device. losa_select_noalloc serves them: it runs the same three selection kernels as losa_select,
+// but their scratch (the per-row staging lists and the per-row counts) lives in the fixed device array below, which
+// every GPU that loads this library holds until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_select_scratch on the current device. In host code the array's name only stands in for the
+// symbol; the address a kernel can use comes from cudaGetSymbolAddress, looked up once per device with that device
+// current (the lookup may load this library's device code onto the device).
+void* scratch_on_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
+        g_scratch_ptr[dev] = p;
+    }
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" losa_status losa_select_noalloc(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
+                                           int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order,
+                                           cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_INVALID_ARG;
+    if (!aligned16(mass) || !indptr || !kv_block_idx || !order) return LOSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
+         reinterpret_cast<uintptr_t>(order)) & 3u)
+        return LOSA_ERR_INVALID_ARG;
+    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
+    const long long rows = (long long)shape->heads * nq;
+    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
+    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
+    // The fixed scratch must hold rows * nk staged indices plus rows counts.
+    if (select_ws_bytes(shape) > kNoAllocScratchBytes) return LOSA_ERR_CAPACITY;
+
+    void* scratch = scratch_on_current_device();
+    if (!scratch) return LOSA_ERR_CUDA;
+    // Both scratch regions are fully written before they are read, so stale contents from an earlier call need
+    // no clearing.
+    int32_t* staged = static_cast<int32_t*>(scratch);
+    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
+    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(scratch) + staged_bytes);
+
+    const int n2 = next_pow2(nk);
+    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
+    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem1) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, counts,
+                                                                                         staged);
+    if ((st = launch_status()) != LOSA_OK) return st;
+    const int r2 = next_pow2((int)rows);
+    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
+    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem2) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
+    if ((st = launch_status()) != LOSA_OK) return st;
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
+    return launch_status();
+}

@@ -8,7 +8,8 @@
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is DEVICE memory owned by the caller (allocated on the current device). The
- *     library allocates nothing and keeps no state between calls other than one per-device error word.
+ *     library allocates nothing and keeps no state between calls other than one per-device error word (and the
+ *     fixed scratch array of losa_select_noalloc).
  *   - Every call is asynchronous and stream-ordered on `stream`, except losa_get_device_error (which
  *     synchronises the stream). Host-side argument checks run first and return before anything is launched.
  *   - Token tensors q, k, v, o are [H][Np][d] row-major, d contiguous: head h, token t starts at element
@@ -96,6 +97,23 @@ losa_status losa_select(const losa_shape* shape, const float* mass, double tau, 
 
 /* Bytes of device workspace losa_select needs for this shape (0 if the shape is invalid). */
 size_t losa_select_workspace_bytes(const losa_shape* shape);
+
+/*
+ * losa_select without a workspace argument, for callers that cannot allocate device memory when they call: for
+ * example a server that reserved almost all device memory for its own pool at start-up, a plugin whose host
+ * framework owns every buffer, or a latency-critical path where cudaMalloc / cudaFree may synchronise the device.
+ * The pages have no counterpart of this entry point; it exists for such callers only.
+ *   Arguments and results are those of losa_select (same kernels, same output, bit for bit); there is no workspace.
+ *   Scratch: a fixed 16 MiB device array inside the library, present on every GPU that loads it until the process
+ *   exits. Shapes whose scratch need (losa_select_workspace_bytes) exceeds 16 MiB return LOSA_ERR_CAPACITY: that
+ *   admits H * nq * nk up to about 4.1 million (a 12-head layer of 256 x 256 blocks needs 3.2 MB).
+ *   The library allocates nothing in this call. Its first call on a device looks up the array's device address
+ *   (which may load the library's device code onto that device), so make that first call before any stream capture.
+ *   Every call on a device shares the one array and overwrites what the previous call left there: calls whose GPU
+ *   work can overlap (different streams without ordering between them) race on it and must be serialised.
+ */
+losa_status losa_select_noalloc(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
+                                int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, cudaStream_t stream);
 
 /*
  * Block-sparse attention over a frozen pattern (LoSA page, Methodology Summary, "Sparse attention with a frozen
