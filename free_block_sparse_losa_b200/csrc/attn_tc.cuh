@@ -1,25 +1,30 @@
-// Tensor-core (tcgen05 / TMEM / TMA) attention kernels for bf16 inputs, head_dim 128, 128 x 128 blocks.
+// Tensor-core (tcgen05 / TMEM / TMA) attention kernel for bf16 inputs, head_dim 128, 128 x 128 blocks.
 //
-// One kernel template, two modes:
-//   Fwd  — online-softmax attention of one 128-row query block against a list of 128-key blocks: the full list
-//          0..nk-1 for the dense step (LoSA page, Motivation Summary: A = softmax(Q K^T / sqrt(d))), or the frozen
-//          retained list for the sparse steps (Methodology Summary, "Sparse attention with a frozen pattern":
-//          the softmax denominator covers the retained keys only). Writes O (bf16) and the row log-sum-exp.
-//   Mass — recomputes S = Q K^T for every key block and sums exp(s - lse) with the forward pass's log-sum-exp into
-//          one value per (query block, key block), divided by the block's real rows (Motivation Summary: block
-//          attention mass M(i, j)). The probability matrix is never written to memory.
+// attn_tc_kernel<WITH_MASS> processes work items = (head, 128-row query block):
+//   forward phase — online-softmax attention against a list of 128-key blocks: the full list 0..nk-1 for a dense
+//                   step (LoSA page, Motivation Summary: A = softmax(Q K^T / sqrt(d))) or the frozen retained list for
+//                   later steps (Methodology Summary, "Sparse attention with a frozen pattern": the softmax
+//                   denominator covers the retained keys only). Writes O (bf16) and the row log-sum-exp.
+//   mass phase    — (WITH_MASS) recomputes S = Q K^T for every key block and sums 2^(s*c - lse2) with the forward
+//                   phase's exact log-sum-exp, still in registers, into one value per (query block, key block), then
+//                   divides by the block's real rows (Motivation Summary: block attention mass M(i, j)). The
+//                   probability matrix is never stored.
 //
-// Persistent grid (one CTA per SM). CTA b takes work items b, 2G-1-b, 2G+b, ... of the item order (a snake over
-// the longest-first order balances list lengths across CTAs). Warp roles inside a CTA (256 threads):
-//   warp 0       TMA producer: Q tile once per item, K/V tiles into a 2-stage ring.
-//   warp 1       MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers, then O += P V into TMEM.
-//                Also owns the TMEM allocation.
-//   warps 4..7   softmax / epilogue: thread t owns query row t (TMEM lane t). Reads S from TMEM, keeps the running
-//                max and sum in registers, writes P (bf16) to shared memory in the 128-byte-swizzled K-major layout
-//                the tensor core reads, and rescales O in TMEM only when a row's max grows by more than 2^8 (the
-//                final division by the row sum makes the choice of reference max exact). Epilogue: O / l -> bf16.
-// Every wait is bounded in time; on expiry the kernel records LOSA_ERR_TIMEOUT in the device error word, waits for
-// its own copies and MMAs in flight, frees TMEM and exits.
+// Persistent grid, one CTA (384 threads) per SM, split into two independent LANES that share the SM's tensor core
+// and TMA unit. Lane x owns 96 KB of shared memory (Q, K and V tiles), 256 TMEM columns (S/P and O, 128 each) and
+// three roles: a TMA producer thread (warp 2x), an MMA issuer thread (warp 2x + 1) and a softmax warpgroup (warps
+// 4 + 4x .. 7 + 4x; thread t owns query row t = TMEM lane t). Lane x takes rounds x, x + 2, x + 4, ... of the CTA's
+// items; CTA b's round r is item r*G + b (r even) or r*G + G - 1 - b (r odd) of the work order, a snake over the
+// longest-first order. Inside a lane, tile t flows QK^T -> softmax -> P V -> next QK^T; the other lane fills the
+// tensor core meanwhile, and two softmax warps per SM sub-partition hide each other's latencies.
+//
+// S = Q K^T lands in the lane's S/P columns; the softmax writes P = 2^(s*c - m*c) as packed bf16 into the first 64
+// of them and the MMA computes O += P V with P read from TMEM (V is an MN-major shared-memory operand). O is
+// rescaled in place only when a row's running max grows by more than 2^8 (the final division by the sum taken
+// against the same reference keeps this exact).
+//
+// Every wait is bounded in time; on expiry the kernel records LOSA_ERR_TIMEOUT in the device error word, waits for its
+// own copies and MMAs in flight, frees TMEM and exits.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -27,33 +32,23 @@
 
 namespace losa {
 
-enum class TcMode : int { Fwd = 0, Mass = 1 };
-
 constexpr int kTcRows = 128;      // R = C = 128
 constexpr int kTcDim = 128;       // head_dim
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
 constexpr uint32_t kTileBytes = kTcRows * kTcDim * 2;   // 32 KB: one 128 x 128 bf16 tile
 constexpr uint32_t kBoxBytes = kTileBytes / 2;         // 16 KB: one 128-row x 64-column TMA box
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;  // bound of the exit-path waits
+constexpr int kMaxMassBlocks = 1024;                   // nk limit of the mass phase (partial-sum buffer)
 
-// Shared-memory map (offsets from a 1024-byte-aligned base).
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;            // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;        // 2 stages (Fwd)
-constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;        // Fwd
-constexpr uint32_t kOffPart = kOffV;                      // Mass: 2 x [4][1024] fp32 partial sums (nk <= 1024)
-constexpr uint32_t kPartFloats = 4 * 1024;
-constexpr uint32_t kFwdBarOff = kOffP + kTileBytes;
-constexpr uint32_t kMassBarOff = kOffPart + 2 * kPartFloats * 4;
-constexpr uint32_t kBarBytes = 256;
-constexpr uint32_t tc_smem_bytes(TcMode m) {
-    return (m == TcMode::Fwd ? kFwdBarOff : kMassBarOff) + kBarBytes + 1024;  // + alignment slack
+// Per-lane shared memory (from a 1024-aligned base): Q, K, V tiles, then (mass) 4 x 1024 fp32 partial sums.
+constexpr uint32_t kLaneQ = 0, kLaneK = kTileBytes, kLaneV = 2 * kTileBytes;
+constexpr uint32_t kLaneTiles = 3 * kTileBytes;                         // 96 KB
+constexpr uint32_t kPartBytes = 4 * kMaxMassBlocks * 4;                 // 16 KB
+constexpr uint32_t kBarBytes = 256;                                     // per lane
+template <bool M>
+constexpr uint32_t tc_smem_bytes() {
+    return 2 * kLaneTiles + (M ? 2 * kPartBytes : 0) + 2 * kBarBytes + 1024;  // + alignment slack
 }
-
-// Barrier slots (8 bytes each).
-enum : uint32_t {
-    B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_K_EMPTY = 4, B_V_FULL = 6, B_V_EMPTY = 8, B_S_FULL = 10,
-    B_S_FREE = 12, B_P_FULL = 14, B_O_READY = 15, B_O_FREE = 16, B_MMA_DONE = 17, B_PART = 18, B_COUNT = 19
-};
 
 struct TcArgs {
     int H, N, Np, nq, nk, n_items;
@@ -61,9 +56,9 @@ struct TcArgs {
     const int32_t* indptr;         // null: dense list 0..nk-1
     const int32_t* kv_idx;
     const int32_t* order;          // null: ascending item ids
-    __nv_bfloat16* o;              // Fwd output
-    float* lse;                    // Fwd: output (may be null); Mass: input
-    float* mass;                   // Mass output [n_items... H*nq][nk]
+    __nv_bfloat16* o;
+    float* lse;                    // may be null
+    float* mass;                   // [H*nq][nk], WITH_MASS only
     unsigned long long wait_limit_ns;
 };
 
@@ -90,7 +85,8 @@ struct ItemInfo {
     int id, h, qb, begin, count;
 };
 
-__device__ __forceinline__ bool next_item(const TcArgs& a, int round, ItemInfo& it) {
+// Item of CTA round `round` (false past the end of the work order).
+__device__ __forceinline__ bool item_of_round(const TcArgs& a, int round, ItemInfo& it) {
     const int G = gridDim.x, b = blockIdx.x;
     const long long w = (long long)round * G + ((round & 1) ? (G - 1 - b) : b);
     if (w >= a.n_items) return false;
@@ -107,13 +103,69 @@ __device__ __forceinline__ bool next_item(const TcArgs& a, int round, ItemInfo& 
     return true;
 }
 
-__device__ __forceinline__ int tile_block(const TcArgs& a, const ItemInfo& it, int t) {
+// Key block of forward tile t (the producer reports out-of-range indices; everyone uses the clamped value).
+__device__ __forceinline__ int fwd_block(const TcArgs& a, const ItemInfo& it, int t) {
     if (!a.indptr) return t;
     const int j = a.kv_idx[it.begin + t];
-    return (j < 0) ? 0 : (j >= a.nk ? a.nk - 1 : j);  // out-of-range indices are reported by the producer
+    return (j < 0) ? 0 : (j >= a.nk ? a.nk - 1 : j);
 }
 
-template <TcMode MODE>
+// 2^x on the FMA/ALU pipes, to take part of the load off the exp unit. Cody-Waite split x = n + f with n = round(x)
+// (the 1.5 * 2^23 shift leaves n in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial whose
+// coefficients minimise the maximum relative error on that interval (fitted by Lawson's iteratively reweighted least
+// squares; max relative error 2.7e-6 evaluated in fp32 Horner form); n is added to the exponent field. Valid for
+// x <= 126; inputs below -125 are clamped there (2^-125 ~ 2.4e-38), so callers that need exact zeros (masked keys)
+// use ex2_approx instead.
+constexpr float kExp2C0 = 0.9999992847442627f, kExp2C1 = 0.6931217908859253f, kExp2C2 = 0.240247443318367f,
+                kExp2C3 = 0.05591785907745361f, kExp2C4 = 0.009570102207362652f;
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(kExp2C4, f, kExp2C3);
+    p = fmaf(p, f, kExp2C2);
+    p = fmaf(p, f, kExp2C1);
+    p = fmaf(p, f, kExp2C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// exp2_poly on a pair of fp32 values with packed f32x2 arithmetic (the integer exponent update stays scalar).
+__device__ __forceinline__ void exp2_poly2(uint64_t xx, float& r0, float& r1) {
+    float x0, x1;
+    f2_unpack(xx, x0, x1);
+    xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = f2_add(xx, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), xx);
+    uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+    p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T: the A operand (P) is read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Barrier slots of one lane (8 bytes each). Counts: P_FULL, O_FREE, S_FREE, PART take 128 arrivals, the rest 1.
+enum : uint32_t {
+    L_Q_FULL = 0, L_Q_EMPTY, L_K_FULL, L_K_EMPTY, L_V_FULL, L_V_EMPTY, L_S_FULL, L_P_FULL, L_PV_DONE, L_O_FREE,
+    L_S_FREE, L_PART, L_MMA_DONE, L_COUNT
+};
+
+template <bool WITH_MASS>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -121,305 +173,374 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const base_ptr = smem_raw + (base - raw);
-    const uint32_t bar0 = base + (MODE == TcMode::Fwd ? kFwdBarOff : kMassBarOff);
-    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + (bar0 - base) + B_COUNT * 8);
-    auto BAR = [&](uint32_t slot) { return bar0 + slot * 8u; };
-    constexpr uint32_t kTmemCols = (MODE == TcMode::Fwd) ? 512u : 256u;
+    const uint32_t part_off = 2 * kLaneTiles;
+    const uint32_t bar_off = part_off + (WITH_MASS ? 2 * kPartBytes : 0);
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + bar_off + 2 * kBarBytes - 16);
 
     const int warp = threadIdx.x >> 5;
     const uint32_t lane = lane_id();
+    // lane x: producer warp 2x, MMA warp 2x + 1, softmax warps 4 + 4x .. 7 + 4x
+    const uint32_t x = (warp < 4) ? (uint32_t)(warp >> 1) : (uint32_t)((warp - 4) >> 2);
+    const uint32_t bar0 = base + bar_off + x * kBarBytes;
+    auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
+    const uint32_t sQ = base + x * kLaneTiles + kLaneQ;
+    const uint32_t sK = base + x * kLaneTiles + kLaneK;
+    const uint32_t sV = base + x * kLaneTiles + kLaneV;
 
-    if (threadIdx.x == 0) {
-        mbar_init(BAR(B_Q_FULL), 1);
-        mbar_init(BAR(B_Q_EMPTY), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(BAR(B_K_FULL + s), 1);
-            mbar_init(BAR(B_K_EMPTY + s), 1);
-            mbar_init(BAR(B_V_FULL + s), 1);
-            mbar_init(BAR(B_V_EMPTY + s), 1);
-            mbar_init(BAR(B_S_FULL + s), 1);
-            mbar_init(BAR(B_S_FREE + s), 128);
+    if (threadIdx.x < 2) {  // thread 0 initialises lane 0's barriers, thread 1 lane 1's
+        const uint32_t b0 = base + bar_off + threadIdx.x * kBarBytes;
+        for (uint32_t s = 0; s < L_COUNT; ++s) {
+            const bool wide = (s == L_P_FULL || s == L_O_FREE || s == L_S_FREE || s == L_PART);
+            mbar_init(b0 + 8u * s, wide ? 128u : 1u);
         }
-        mbar_init(BAR(B_P_FULL), 128);
-        mbar_init(BAR(B_O_READY), 1);
-        mbar_init(BAR(B_O_FREE), 128);
-        mbar_init(BAR(B_MMA_DONE), 1);
-        mbar_init(BAR(B_PART), 128);
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_alloc(smem_addr(tmem_slot), 512);
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
-        if (MODE == TcMode::Fwd) tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmV);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+    const uint32_t tS = tmem + x * 256u;        // lane's S/P columns
+    const uint32_t tO = tS + 128u;              // lane's O columns
     const unsigned long long lim = a.wait_limit_ns;
+    const int mass_tiles = WITH_MASS ? a.nk : 0;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------------------ TMA producer
+    if (warp < 4 && (warp & 1) == 0) {
+        // ------------------------------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t kc = 0, nq_loads = 0;
-            uint32_t nk_loads[2] = {0u, 0u}, nv_loads[2] = {0u, 0u};
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            uint32_t nq = 0, nk_ld = 0, nv_ld = 0;
             bool ok = true;
             ItemInfo it;
-            for (int round = 0; ok && next_item(a, round, it); ++round) {
+            for (int r = (int)x; ok && item_of_round(a, r, it); r += 2) {
                 if (it.count <= 0) {
                     if (a.indptr) atomicOr(&g_device_error, kDevErrBadData);
                     continue;
                 }
-                if (!(ok = wait_bounded(BAR(B_Q_EMPTY), (nq_loads & 1u) ^ 1u, lim))) break;
+                if (!(ok = wait_bounded(BAR(L_Q_EMPTY), (nq & 1u) ^ 1u, lim))) break;
                 const int32_t qrow = it.h * a.Np + it.qb * kTcRows;
-                mbar_arrive_expect_tx(BAR(B_Q_FULL), kTileBytes);
-                tma_load_2d(base + kOffQ, &tmQ, 0, qrow, BAR(B_Q_FULL));
-                tma_load_2d(base + kOffQ + kBoxBytes, &tmQ, 64, qrow, BAR(B_Q_FULL));
-                ++nq_loads;
-                for (int t = 0; t < it.count; ++t, ++kc) {
-                    if (a.indptr) {
+                mbar_arrive_expect_tx(BAR(L_Q_FULL), kTileBytes);
+                tma_load_2d_hint(sQ, &tmQ, 0, qrow, BAR(L_Q_FULL), pol_q);
+                tma_load_2d_hint(sQ + kBoxBytes, &tmQ, 64, qrow, BAR(L_Q_FULL), pol_q);
+                ++nq;
+                const int total = it.count + mass_tiles;
+                int jn = fwd_block(a, it, 0);  // block index fetched one tile ahead
+                for (int t = 0; t < total; ++t) {
+                    const bool fwd = t < it.count;
+                    const int j = jn;
+                    if (t + 1 < it.count) jn = fwd_block(a, it, t + 1);
+                    else jn = t + 1 - it.count;  // mass phase: every block in order
+                    if (fwd && a.indptr) {
                         const int jr = a.kv_idx[it.begin + t];
                         if (jr < 0 || jr >= a.nk) atomicOr(&g_device_error, kDevErrBadData);
                     }
-                    const int32_t krow = it.h * a.Np + tile_block(a, it, t) * kTcRows;
-                    const uint32_t s = kc & 1u, ph = (kc >> 1) & 1u;
-                    if (!(ok = wait_bounded(BAR(B_K_EMPTY + s), ph ^ 1u, lim))) break;
-                    mbar_arrive_expect_tx(BAR(B_K_FULL + s), kTileBytes);
-                    tma_load_2d(base + kOffK + s * kTileBytes, &tmK, 0, krow, BAR(B_K_FULL + s));
-                    tma_load_2d(base + kOffK + s * kTileBytes + kBoxBytes, &tmK, 64, krow, BAR(B_K_FULL + s));
-                    ++nk_loads[s];
-                    if (MODE == TcMode::Fwd) {
-                        if (!(ok = wait_bounded(BAR(B_V_EMPTY + s), ph ^ 1u, lim))) break;
-                        mbar_arrive_expect_tx(BAR(B_V_FULL + s), kTileBytes);
-                        tma_load_2d(base + kOffV + s * kTileBytes, &tmV, 0, krow, BAR(B_V_FULL + s));
-                        tma_load_2d(base + kOffV + s * kTileBytes + kBoxBytes, &tmV, 64, krow, BAR(B_V_FULL + s));
-                        ++nv_loads[s];
+                    const int32_t krow = it.h * a.Np + j * kTcRows;
+                    if (!(ok = wait_bounded(BAR(L_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
+                    mbar_arrive_expect_tx(BAR(L_K_FULL), kTileBytes);
+                    tma_load_2d_hint(sK, &tmK, 0, krow, BAR(L_K_FULL), pol_kv);
+                    tma_load_2d_hint(sK + kBoxBytes, &tmK, 64, krow, BAR(L_K_FULL), pol_kv);
+                    ++nk_ld;
+                    if (fwd) {
+                        if (!(ok = wait_bounded(BAR(L_V_EMPTY), (nv_ld & 1u) ^ 1u, lim))) break;
+                        mbar_arrive_expect_tx(BAR(L_V_FULL), kTileBytes);
+                        tma_load_2d_hint(sV, &tmV, 0, krow, BAR(L_V_FULL), pol_kv);
+                        tma_load_2d_hint(sV + kBoxBytes, &tmV, 64, krow, BAR(L_V_FULL), pol_kv);
+                        ++nv_ld;
                     }
                 }
             }
-            // Drain: wait until every copy this thread issued has landed (they complete on their own).
-            if (nq_loads) wait_bounded(BAR(B_Q_FULL), (nq_loads - 1) & 1u, lim);
-            for (uint32_t s = 0; s < 2; ++s) {
-                if (nk_loads[s]) wait_bounded(BAR(B_K_FULL + s), (nk_loads[s] - 1) & 1u, lim);
-                if (nv_loads[s]) wait_bounded(BAR(B_V_FULL + s), (nv_loads[s] - 1) & 1u, lim);
-            }
+            // Drain: every copy this thread issued lands before the CTA may exit.
+            if (nq) wait_bounded(BAR(L_Q_FULL), (nq - 1) & 1u, kDrainLimitNs);
+            if (nk_ld) wait_bounded(BAR(L_K_FULL), (nk_ld - 1) & 1u, kDrainLimitNs);
+            if (nv_ld) wait_bounded(BAR(L_V_FULL), (nv_ld - 1) & 1u, kDrainLimitNs);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------------------ MMA issuer
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t kIdPV = idesc_bf16_f32(128, 128, false, true);
-            uint32_t kc = 0, items = 0, pc = 0;
+            uint32_t nq = 0, nk_use = 0, nv_use = 0, n_pv = 0, n_sfree = 0, n_items = 0;
             bool ok = true;
-            bool pend = false;
-            uint32_t p_s = 0, p_ph = 0, p_first = 0, p_item = 0;
-            auto issue_pv = [&]() -> bool {
-                if (!wait_bounded(BAR(B_P_FULL), pc & 1u, lim)) return false;
-                if (!wait_bounded(BAR(B_V_FULL + p_s), p_ph, lim)) return false;
-                if (p_first && !wait_bounded(BAR(B_O_FREE), (p_item & 1u) ^ 1u, lim)) return false;
-                tc_fence_after();
-                const uint32_t vbase = base + kOffV + p_s * kTileBytes;
-#pragma unroll
-                for (uint32_t kk = 0; kk < 8; ++kk) {
-                    const uint64_t da = smem_desc(base + kOffP + (kk >> 2) * kBoxBytes + (kk & 3u) * 32u, 16, 1024);
-                    const uint64_t db = smem_desc(vbase + kk * 2048u, kBoxBytes, 1024);
-                    tc_mma_ss(tmem + 256u, da, db, kIdPV, (p_first && kk == 0) ? 0u : 1u);
-                }
-                tc_commit(BAR(B_V_EMPTY + p_s));
-                tc_commit(BAR(B_O_READY));
-                ++pc;
-                return true;
-            };
             ItemInfo it;
-            for (int round = 0; ok && next_item(a, round, it); ++round) {
+            for (int r = (int)x; ok && item_of_round(a, r, it); r += 2) {
                 if (it.count <= 0) continue;
-                if (!(ok = wait_bounded(BAR(B_Q_FULL), items & 1u, lim))) break;
-                tc_fence_after();
-                for (int t = 0; t < it.count; ++t, ++kc) {
-                    const uint32_t s = kc & 1u, ph = (kc >> 1) & 1u;
-                    if (!(ok = wait_bounded(BAR(B_K_FULL + s), ph, lim))) break;
-                    if (!(ok = wait_bounded(BAR(B_S_FREE + s), ph ^ 1u, lim))) break;
+                if (!(ok = wait_bounded(BAR(L_Q_FULL), nq & 1u, lim))) break;
+                ++nq;
+                const int total = it.count + mass_tiles;
+                for (int t = 0; t < total; ++t) {
+                    const bool fwd = t < it.count;
+                    if (!(ok = wait_bounded(BAR(L_K_FULL), nk_use & 1u, lim))) break;
+                    // The S/P columns are free once the previous tile's P V (forward) or S read (mass) completed.
+                    if (t > 0 && t <= it.count) {
+                        if (!(ok = wait_bounded(BAR(L_PV_DONE), (n_pv - 1) & 1u, lim))) break;
+                    } else if (t > it.count) {
+                        if (!(ok = wait_bounded(BAR(L_S_FREE), (n_sfree - 1) & 1u, lim))) break;
+                    } else if (n_items > 0) {
+                        // first tile of an item: the previous item's last S/P use must be over
+                        if (!(ok = (mass_tiles ? wait_bounded(BAR(L_S_FREE), (n_sfree - 1) & 1u, lim)
+                                               : wait_bounded(BAR(L_PV_DONE), (n_pv - 1) & 1u, lim))))
+                            break;
+                    }
                     tc_fence_after();
-                    const uint32_t kbase = base + kOffK + s * kTileBytes;
 #pragma unroll
                     for (uint32_t kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3u) * 32u;
-                        tc_mma_ss(tmem + s * 128u, smem_desc(base + kOffQ + off, 16, 1024),
-                                  smem_desc(kbase + off, 16, 1024), kIdQK, kk ? 1u : 0u);
+                        tc_mma_ss(tS, smem_desc(sQ + off, 16, 1024), smem_desc(sK + off, 16, 1024), kIdQK,
+                                  kk ? 1u : 0u);
                     }
-                    tc_commit(BAR(B_S_FULL + s));
-                    tc_commit(BAR(B_K_EMPTY + s));
-                    if (t == it.count - 1) tc_commit(BAR(B_Q_EMPTY));
-                    if (MODE == TcMode::Fwd) {
-                        if (pend && !(ok = issue_pv())) break;
-                        pend = true;
-                        p_s = s;
-                        p_ph = ph;
-                        p_first = (t == 0);
-                        p_item = items;
+                    tc_commit(BAR(L_S_FULL));
+                    tc_commit(BAR(L_K_EMPTY));
+                    ++nk_use;
+                    if (t == total - 1) tc_commit(BAR(L_Q_EMPTY));
+                    if (fwd) {
+                        if (!(ok = wait_bounded(BAR(L_P_FULL), n_pv & 1u, lim))) break;
+                        if (!(ok = wait_bounded(BAR(L_V_FULL), nv_use & 1u, lim))) break;
+                        if (t == 0 && !(ok = wait_bounded(BAR(L_O_FREE), (n_items & 1u) ^ 1u, lim))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (uint32_t kk = 0; kk < 8; ++kk) {
+                            const uint64_t db = smem_desc(sV + kk * 2048u, kBoxBytes, 1024);
+                            tc_mma_ts(tO, tS + kk * 8u, db, kIdPV, (t == 0 && kk == 0) ? 0u : 1u);
+                        }
+                        tc_commit(BAR(L_V_EMPTY));
+                        tc_commit(BAR(L_PV_DONE));
+                        ++nv_use;
+                        ++n_pv;
+                    } else {
+                        ++n_sfree;  // the softmax frees S after reading it; the wait happens before the next QK
                     }
                 }
-                ++items;
+                ++n_items;
             }
-            if (MODE == TcMode::Fwd && ok && pend) issue_pv();
-            tc_commit(BAR(B_MMA_DONE));
-            wait_bounded(BAR(B_MMA_DONE), 0, lim);
+            tc_commit(BAR(L_MMA_DONE));
+            wait_bounded(BAR(L_MMA_DONE), 0, kDrainLimitNs);
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------------------------ softmax / epilogue
+    } else {
+        // ------------------------------------------------------------------------------- softmax / epilogue
         const uint32_t wl = (uint32_t)warp & 3u;
         const int row = (int)(wl * 32u + lane);
         const uint32_t lane_off = (wl * 32u) << 16;
-        float* const part = reinterpret_cast<float*>(base_ptr + kOffPart);
-        uint32_t kc = 0, oc = 0, done_items = 0;
+        const float c = a.scale_log2;
+        float* const part = reinterpret_cast<float*>(base_ptr + part_off + x * kPartBytes);
+        uint32_t n_s = 0, n_pv = 0, n_items = 0;
         bool ok = true;
         ItemInfo it;
-        for (int round = 0; ok && next_item(a, round, it); ++round) {
+        for (int r = (int)x; ok && item_of_round(a, r, it); r += 2) {
             if (it.count <= 0) continue;
-            float* const pbuf = part + (done_items & 1u) * kPartFloats;
             const int qrow = it.qb * kTcRows + row;
             const size_t grow = (size_t)it.h * a.Np + qrow;
-            float m_run = -INFINITY, l_run = 0.0f, lse2 = 0.0f;
-            const bool qvalid = qrow < a.N;
-            if (MODE == TcMode::Mass) lse2 = qvalid ? a.lse[grow] * 1.4426950408889634f : 0.0f;
-            for (int t = 0; t < it.count; ++t, ++kc) {
-                const uint32_t s = kc & 1u, ph = (kc >> 1) & 1u;
-                if (!(ok = wait_bounded_warp(BAR(B_S_FULL + s), ph, lim))) break;
+            float m_raw = -INFINITY, l_run = 0.0f;
+            int jn = fwd_block(a, it, 0);
+            for (int t = 0; t < it.count; ++t) {
+                const int j = jn;
+                if (t + 1 < it.count) jn = fwd_block(a, it, t + 1);  // prefetch the next block index
+                if (!(ok = wait_bounded_warp(BAR(L_S_FULL), n_s & 1u, lim))) break;
+                ++n_s;
                 tc_fence_after();
-                uint32_t sr[128];
+                const int kvalid = a.N - j * kTcRows;  // < 128 only in the ragged last key block
+                // Pass 1: the tile's row max over all 128 columns (only columns 0..31 stay live afterwards).
+                float s0[32];
+                float tmax;
+                {
+                    float s[128];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]);
-                    tmem_ld32(tmem + lane_off + s * 128u + c * 32u, chunk);
-                }
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(BAR(B_S_FREE + s));
-                const int j = tile_block(a, it, t);
-                const int kvalid = min(kTcRows, a.N - j * kTcRows);
-                if (MODE == TcMode::Mass) {
-                    float sum = 0.0f;
+                    for (int ch = 0; ch < 4; ++ch)
+                        tmem_ld32(tS + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
+                    tmem_wait_ld();
+                    if (kvalid < kTcRows) {  // keys t >= N do not exist
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const float p = ex2_approx(fmaf(__uint_as_float(sr[c]), a.scale_log2, -lse2));
-                        sum += (c < kvalid) ? p : 0.0f;
+                        for (int cc = 0; cc < 128; ++cc)
+                            if (cc >= kvalid) s[cc] = -INFINITY;
                     }
+                    float mx[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+#pragma unroll
+                    for (int cc = 24; cc < 128; cc += 16)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], s[cc + e], s[cc + 8 + e]);
+                    tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s0[e] = s[e];
+                }
+                // Reference max: raised only when the tile max exceeds it by more than 2^8 in the exp2 domain.
+                const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
+                const float alpha = (t > 0 && need) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
+                if (need) m_raw = tmax;
+                const float neg_mc = -m_raw * c;
+                // Pass 2, 32 columns at a time, the next chunk's TMEM load in flight during this chunk's math:
+                // P = 2^(s*c - m*c) as bf16 pairs written behind the read position (columns 16*ch .. 16*ch + 15
+                // hold keys 32*ch .. 32*ch + 31).
+                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                float rb[2][32];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    if (ch < 3)
+                        tmem_ld32(tS + lane_off + (ch + 1) * 32u, *reinterpret_cast<uint32_t(*)[32]>(&rb[(ch + 1) & 1][0]));
+                    const float* r = (ch == 0) ? s0 : rb[ch & 1];
+                    uint32_t pw[16];
+                    if (kvalid >= kTcRows) {
+                        // three pairs in eight on the FMA pipe (packed polynomial), the rest on the exp unit
+                        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t xx = f2_fma(f2_pack(r[2 * e], r[2 * e + 1]), c2, nm2);
+                            float p0, p1;
+                            if ((e & 7) >= 5) {
+                                exp2_poly2(xx, p0, p1);
+                            } else {
+                                float x0, x1;
+                                f2_unpack(xx, x0, x1);
+                                p0 = ex2_approx(x0);
+                                p1 = ex2_approx(x1);
+                            }
+                            pw[e] = pack_bf16x2(p0, p1);
+                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int c0 = ch * 32 + 2 * e;
+                            const float p0 = (c0 < kvalid) ? ex2_approx(fmaf(r[2 * e], c, neg_mc)) : 0.0f;
+                            const float p1 = (c0 + 1 < kvalid) ? ex2_approx(fmaf(r[2 * e + 1], c, neg_mc)) : 0.0f;
+                            pw[e] = pack_bf16x2(p0, p1);
+                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        }
+                    }
+                    tmem_st16(tS + lane_off + ch * 16u, pw);
+                    if (ch < 3) tmem_wait_ld_regs(rb[(ch + 1) & 1]);
+                }
+                float la, lb, lc, ld;
+                f2_unpack(l2[0], la, lb);
+                f2_unpack(l2[1], lc, ld);
+                l_run = l_run * alpha + ((la + lb) + (lc + ld));
+                // O (complete: this tile's S was computed after the previous P V finished) is rescaled before the
+                // P V of this tile may start.
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + lane_off + ch * 32u, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st32(tO + lane_off + ch * 32u, ov);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(L_P_FULL));
+            }
+            if (!ok) break;
+            // Epilogue: O / l -> bf16 rows and lse; O's columns are then free for the next item.
+            if (!(ok = wait_bounded_warp(BAR(L_PV_DONE), (n_pv + it.count - 1) & 1u, lim))) break;
+            n_pv += it.count;
+            tc_fence_after();
+            const float inv_l = 1.0f / l_run;
+            const float lse2 = m_raw * c + lg2_approx(l_run);
+            uint4* dst = reinterpret_cast<uint4*>(a.o + grow * kTcDim);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t ov[32];
+                tmem_ld32(tO + lane_off + ch * 32u, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 0]) * inv_l, __uint_as_float(ov[q4 * 8 + 1]) * inv_l);
+                    v.y = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 2]) * inv_l, __uint_as_float(ov[q4 * 8 + 3]) * inv_l);
+                    v.z = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 4]) * inv_l, __uint_as_float(ov[q4 * 8 + 5]) * inv_l);
+                    v.w = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 6]) * inv_l, __uint_as_float(ov[q4 * 8 + 7]) * inv_l);
+                    dst[ch * 4 + q4] = v;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(L_O_FREE));
+            if (a.lse) a.lse[grow] = lse2 * 0.6931471805599453f;
+
+            if (WITH_MASS) {
+                // Mass phase: p = 2^(s*c - lse2) summed per key block for real rows and real keys.
+                const bool qvalid = qrow < a.N;
+                const float neg_lse2 = qvalid ? -lse2 : 0.0f;
+                for (int j = 0; j < a.nk; ++j) {
+                    if (!(ok = wait_bounded_warp(BAR(L_S_FULL), n_s & 1u, lim))) break;
+                    ++n_s;
+                    tc_fence_after();
+                    float s[128];
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        tmem_ld32(tS + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(BAR(L_S_FREE));
+                    const int kvalid = a.N - j * kTcRows;
+                    uint64_t acc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                    const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(neg_lse2, neg_lse2);
+                    if (kvalid >= kTcRows) {
+                        // seven pairs in sixteen on the FMA pipe (packed polynomial), the rest on the exp unit
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) {
+                            const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nl2);
+                            float p0, p1;
+                            if ((e & 15) >= 9) {
+                                exp2_poly2(xx, p0, p1);
+                            } else {
+                                float x0, x1;
+                                f2_unpack(xx, x0, x1);
+                                p0 = ex2_approx(x0);
+                                p1 = ex2_approx(x1);
+                            }
+                            acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) {
+                            const float p0 = (2 * e < kvalid) ? ex2_approx(fmaf(s[2 * e], c, neg_lse2)) : 0.0f;
+                            const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_lse2)) : 0.0f;
+                            acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+                        }
+                    }
+                    float a0, a1, a2, a3, a4, a5, a6, a7;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], a2, a3);
+                    f2_unpack(acc[2], a4, a5);
+                    f2_unpack(acc[3], a6, a7);
+                    float sum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
                     if (!qvalid) sum = 0.0f;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (lane == 0) pbuf[wl * 1024u + (uint32_t)j] = sum;
-                } else {
-                    float x[128];
-                    float tmax = -INFINITY;
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        x[c] = (c < kvalid) ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
-                        tmax = fmaxf(tmax, x[c]);
-                    }
-                    if (t == 0) {
-                        m_run = tmax;
-                    } else {
-                        // PV of the previous tile must be complete before P is overwritten or O is rescaled.
-                        if (!(ok = wait_bounded_warp(BAR(B_O_READY), oc & 1u, lim))) break;
-                        ++oc;
-                        const bool need = tmax > m_run + 8.0f;
-                        if (__any_sync(0xffffffffu, need)) {
-                            const float alpha = need ? ex2_approx(m_run - tmax) : 1.0f;
-                            tc_fence_after();
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                uint32_t ov[32];
-                                tmem_ld32(tmem + lane_off + 256u + c * 32u, ov);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                                tmem_st32(tmem + lane_off + 256u + c * 32u, ov);
-                            }
-                            tmem_wait_st();
-                            if (need) {
-                                l_run *= alpha;
-                                m_run = tmax;
-                            }
-                        }
-                    }
-                    // P = 2^(x - m_run) in bf16, stored in the 128B-swizzled K-major layout.
-                    const uint32_t prow = base + kOffP + (uint32_t)row * 128u;
-                    float lsum = 0.0f;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                        for (int ch = 0; ch < 8; ++ch) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int c = half * 64 + ch * 8 + e * 2;
-                                const float p0 = ex2_approx(x[c] - m_run);
-                                const float p1 = ex2_approx(x[c + 1] - m_run);
-                                lsum += p0 + p1;
-                                w[e] = pack_bf16x2(p0, p1);
-                            }
-                            const uint32_t addr = prow + (uint32_t)half * kBoxBytes +
-                                                  (uint32_t)((ch ^ (row & 7)) * 16);
-                            st_shared_v4(addr, w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                    l_run += lsum;
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(BAR(B_P_FULL));
+                    if (lane == 0) part[wl * kMaxMassBlocks + j] = sum;
                 }
-            }
-            if (!ok) break;
-            if (MODE == TcMode::Mass) {
-                // All four warps' partial sums of this item are in pbuf once the 128 threads have arrived. The
-                // next item writes the other buffer, and the one after that only starts once every thread has
-                // arrived again, i.e. finished reading this one.
-                mbar_arrive(BAR(B_PART));
-                if (!(ok = wait_bounded_warp(BAR(B_PART), done_items & 1u, lim))) break;
+                if (!ok) break;
+                // The four warps' partial sums are complete once all 128 threads have arrived. The next item's
+                // partials are written only after every thread has passed its forward tiles, i.e. after this read.
+                mbar_arrive(BAR(L_PART));
+                if (!(ok = wait_bounded_warp(BAR(L_PART), n_items & 1u, lim))) break;
                 const float inv_rows = 1.0f / (float)min(kTcRows, a.N - it.qb * kTcRows);
                 float* mrow = a.mass + (size_t)it.id * a.nk;
                 for (int jj = row; jj < a.nk; jj += 128)
-                    mrow[jj] = (pbuf[jj] + pbuf[1024 + jj] + pbuf[2048 + jj] + pbuf[3072 + jj]) * inv_rows;
-            } else {
-                if (!(ok = wait_bounded_warp(BAR(B_O_READY), oc & 1u, lim))) break;
-                ++oc;
-                tc_fence_after();
-                const float inv_l = 1.0f / l_run;
-                __nv_bfloat16* orow = a.o + grow * kTcDim;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t ov[32];
-                    tmem_ld32(tmem + lane_off + 256u + c * 32u, ov);
-                    tmem_wait_ld();
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 0]) * inv_l, __uint_as_float(ov[q4 * 8 + 1]) * inv_l);
-                        v.y = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 2]) * inv_l, __uint_as_float(ov[q4 * 8 + 3]) * inv_l);
-                        v.z = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 4]) * inv_l, __uint_as_float(ov[q4 * 8 + 5]) * inv_l);
-                        v.w = pack_bf16x2(__uint_as_float(ov[q4 * 8 + 6]) * inv_l, __uint_as_float(ov[q4 * 8 + 7]) * inv_l);
-                        dst[q4] = v;
-                    }
-                }
-                if (a.lse) a.lse[grow] = (m_run + lg2_approx(l_run)) * 0.6931471805599453f;
-                tc_fence_before();
-                mbar_arrive(BAR(B_O_FREE));
+                    mrow[jj] = ((part[jj] + part[kMaxMassBlocks + jj]) +
+                                (part[2 * kMaxMassBlocks + jj] + part[3 * kMaxMassBlocks + jj])) * inv_rows;
             }
-            ++done_items;
+            ++n_items;
         }
     }
     // Teardown: every role has left its loop (normally or after a bounded wait ran out).
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace losa

@@ -52,7 +52,7 @@ losa_status check_shape(const losa_shape* s) {
 
 bool tc_shape(const losa_shape* s) {
     return s->dtype == LOSA_DTYPE_BF16 && s->head_dim == kTcDim && s->block_q == kTcRows && s->block_k == kTcRows &&
-           s->n_padded / kTcRows <= 1024;
+           s->n_padded / kTcRows <= kMaxMassBlocks;
 }
 
 bool f32_shape(const losa_shape* s) {
@@ -103,14 +103,14 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <TcMode MODE>
-losa_status launch_tc(const losa_shape* s, const void* q, const void* k, const void* v, float scale,
+// Tensor-core path: fills the argument block and launches one persistent CTA (two lanes) per SM.
+losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const void* k, const void* v, float scale,
                       const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
                       float* mass, cudaStream_t stream) {
     const uint64_t rows = (uint64_t)s->heads * s->n_padded;
     CUtensorMap tq, tk, tv;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows)) return LOSA_ERR_CUDA;
-    if (!make_tile_map(&tv, v ? v : k, rows)) return LOSA_ERR_CUDA;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+        return LOSA_ERR_CUDA;
     TcArgs a;
     a.H = s->heads;
     a.N = s->n_tokens;
@@ -128,12 +128,21 @@ losa_status launch_tc(const losa_shape* s, const void* q, const void* k, const v
     a.wait_limit_ns = g_wait_limit_ns;
     const int sms = sm_count();
     if (sms <= 0) return LOSA_ERR_CUDA;
-    const int grid = a.n_items < sms ? a.n_items : sms;
-    const uint32_t smem = tc_smem_bytes(MODE);
-    if (cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return LOSA_ERR_CUDA;
-    attn_tc_kernel<MODE><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
+    const int want = (a.n_items + 1) / 2;  // two lanes per CTA
+    const int grid = want < sms ? (want > 0 ? want : 1) : sms;
+    if (with_mass) {
+        const uint32_t smem = tc_smem_bytes<true>();
+        if (cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return LOSA_ERR_CUDA;
+        attn_tc_kernel<true><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
+    } else {
+        const uint32_t smem = tc_smem_bytes<false>();
+        if (cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return LOSA_ERR_CUDA;
+        attn_tc_kernel<false><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
+    }
     return launch_status();
 }
 
@@ -221,10 +230,7 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
     if (mass && !aligned16(mass)) return LOSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
     if (tc_shape(shape)) {
-        st = launch_tc<TcMode::Fwd>(shape, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, nullptr, stream);
-        if (st != LOSA_OK || !mass) return st;
-        return launch_tc<TcMode::Mass>(shape, q, k, nullptr, scale, nullptr, nullptr, nullptr, nullptr, lse, mass,
-                                       stream);
+        return launch_tc(shape, mass != nullptr, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, mass, stream);
     }
     if (f32_shape(shape)) {
         if (shape->head_dim == 64)
@@ -291,7 +297,7 @@ losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void*
     if (lse && !aligned16(lse)) return LOSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
     if (tc_shape(shape))
-        return launch_tc<TcMode::Fwd>(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
+        return launch_tc(shape, false, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
     if (f32_shape(shape)) {
         if (shape->head_dim == 64)
             return launch_f32<64>(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse, nullptr, stream);
