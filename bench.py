@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 
 from losa_synth import CONFIGS, make_layer, sample_items  # noqa: E402
 
-WORKLOADS = {"hunyuan720": 3, "wan14b720": 2, "wan1.3b480": 1, "tiny": 0}
+WORKLOADS = {"hunyuan720": 3, "wan14b720": 2, "wan1.3b480": 1, "tiny": 0, "loop": 4}
 METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select ms"
 KERNELS_PER_STEP = {"dense_profile": 2, "select": 3, "sparse_attn": 1}
 
@@ -386,6 +386,115 @@ def run_native(args, cfg):
     return 0
 
 
+# ------------------------------------------------------------------------------------------ reuse loop
+
+def run_loop(args, cfg):
+    """Denoising-loop reuse at the Wan2.1-480p shape: steps before the construction step t0 are dense, step t0
+    profiles every layer and selects its pattern (t0 = 0 by default; the LoSA page's setup uses t0 = 3), later steps
+    run sparse attention with the frozen lists on Q/K/V that drift each step. Each layer's dense call on the same
+    inputs is timed beside it, giving the 50-dense-step baseline. Reports totals, the sampled approximation error
+    of the sparse output against fp64 dense attention, and the recall of the frozen pattern under later steps' exact
+    masses."""
+    import torch
+    import free_block_sparse_losa_b200 as L
+    from free_block_sparse_losa_b200.harness import LayerBuffers
+    from losa_synth import Drift
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    L.load()
+    n_layers = args.loop_layers or cfg.layers
+    n_steps = args.loop_steps or cfg.extra["steps"]
+    layers = [make_layer(cfg, li) for li in range(n_layers)]
+    drift = Drift(cfg, layers, seed=cfg.seed)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    bufs = [LayerBuffers.for_config(cfg) for _ in range(n_layers)]
+    dense_o = torch.empty_like(bufs[0].o)
+    dense_lse = torch.empty_like(bufs[0].lse)
+    probe = LayerBuffers.for_config(cfg)  # dense profile for recall measurements (not timed)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    t_sparse_path, t_dense_path = [], []
+    t0 = args.construct_step
+    report_steps = sorted({t0 + 1, n_steps // 5, n_steps // 2, n_steps - 1} & set(range(t0 + 1, n_steps)))
+    rel_l2, recall = {}, {}
+    items = sample_items(cfg, 8, seed=99)
+    # warm-up of both call kinds on step-0 inputs
+    q, k, v = drift.tokens(0)
+    for _ in range(3):
+        bufs[0].profile(q, k, v, scale)
+        bufs[0].select(args.tau)
+        bufs[0].sparse(q, k, v, scale)
+        L.losa_dense_profile(bufs[0].shape, q, k, v, scale, dense_o, dense_lse, None)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for step in range(n_steps):
+            if step > 0:
+                drift.advance()
+            step_sparse, step_dense = [], []
+            for li in range(n_layers):
+                q, k, v = drift.tokens(li)
+                b = bufs[li]
+                e0, e1, e2 = ev(), ev(), ev()
+                e0.record(stream)
+                if step < t0:
+                    L.losa_dense_profile(b.shape, q, k, v, scale, b.o, b.lse, None)
+                elif step == t0:
+                    b.profile(q, k, v, scale)
+                    b.select(args.tau)
+                else:
+                    b.sparse(q, k, v, scale)
+                e1.record(stream)
+                L.losa_dense_profile(b.shape, q, k, v, scale, dense_o, dense_lse, None)
+                e2.record(stream)
+                step_sparse.append((e0, e1))
+                step_dense.append((e1, e2))
+                if step in report_steps and li == 0:
+                    torch.cuda.synchronize()
+                    qf, kf, vf = (x.float().cpu().numpy() for x in (q, k, v))
+                    ref, _ = oracle.dense(qf, kf, vf, cfg.n_tokens, cfg.block, scale, items)
+                    got = b.o.float().cpu().numpy().reshape(cfg.heads * cfg.n_blocks, cfg.block, cfg.head_dim)
+                    gd = dense_o.float().cpu().numpy().reshape(got.shape)
+                    ok = ~np.isnan(ref)
+                    rel_l2[step] = {"sparse_vs_dense_fp64": float(np.linalg.norm((got[items] - ref)[ok]) /
+                                                                  np.linalg.norm(ref[ok])),
+                                    "dense_kernel_vs_dense_fp64": float(np.linalg.norm((gd[items] - ref)[ok]) /
+                                                                        np.linalg.norm(ref[ok]))}
+                    probe.profile(q, k, v, scale)
+                    m = probe.mass.cpu().numpy().reshape(probe.rows, probe.nk).astype(np.float64)
+                    gi, gk, _ = b.csr_host()
+                    recall[step] = oracle.recall(m, gi, gk)
+            torch.cuda.synchronize()
+            t_sparse_path.append(sum(a.elapsed_time(z) for a, z in step_sparse))
+            t_dense_path.append(sum(a.elapsed_time(z) for a, z in step_dense))
+    if L.losa_get_device_error() != 0:
+        raise RuntimeError("device error in the reuse loop")
+    nnz = [int(b.indptr[-1].item()) for b in bufs]
+    loop_ms, dense_ms = sum(t_sparse_path), sum(t_dense_path)
+    line = {"metric": f"denoising reuse loop ({n_layers} layers x {n_steps} steps): dense steps, profile+select at "
+                      f"step {t0}, then sparse steps, vs dense steps", "value": round(dense_ms / loop_ms, 4),
+            "unit": "x (dense loop time / LoSA loop time)", "n_gpus": 1, "steps": n_steps, "warmup": 3,
+            "ms_per_step": round(loop_ms / n_steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic, drifted 0.02 rms per step",
+            "config": {"workload": cfg.name, "layers": n_layers, "heads": cfg.heads, "n_tokens": cfg.n_tokens,
+                       "head_dim": cfg.head_dim, "block": cfg.block, "tau": args.tau},
+            "loop_ms": round(loop_ms, 3), "dense_loop_ms": round(dense_ms, 3),
+            "construct_step": t0,
+            "construct_step_profile_select_ms": round(t_sparse_path[t0], 3),
+            "construct_step_dense_ms": round(t_dense_path[t0], 3),
+            "sparse_step_ms_mean": round(float(np.mean(t_sparse_path[t0 + 1:])), 3) if n_steps > t0 + 1 else None,
+            "dense_step_ms_mean": round(float(np.mean(t_dense_path)), 3),
+            "block_density": round(sum(nnz) / (n_layers * cfg.heads * cfg.n_blocks ** 2), 5),
+            "rel_l2_layer0_sampled": rel_l2, "recall_of_frozen_pattern_layer0": recall,
+            "gpu_launches": n_layers * (t0 + 1 + 3 + (n_steps - 1 - t0) + n_steps),
+            "clocks": clocks.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -396,11 +505,20 @@ def main():
     ap.add_argument("--tau", type=float, default=0.99)
     ap.add_argument("--cpu-items", type=int, default=0, help="oracle sample size (0: one item per host thread)")
     ap.add_argument("--ref-items", type=int, default=0, help="reference-arm items per step (0: half the threads)")
+    ap.add_argument("--loop-layers", type=int, default=0, help="reuse loop: layers (0: the config's 30)")
+    ap.add_argument("--loop-steps", type=int, default=0, help="reuse loop: denoising steps (0: the config's 50)")
+    ap.add_argument("--construct-step", type=int, default=0, help="reuse loop: step t0 that builds the pattern")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     cfg = CONFIGS[WORKLOADS[args.workload]]
+    if args.workload == "loop":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reuse loop has no CPU-oracle arm; its "
+                              "accuracy is checked against the oracle inside the loop"}))
+            return 0
+        return run_loop(args, cfg)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_native(args, cfg)

@@ -196,3 +196,47 @@ def sample_items(cfg: LayerConfig, n: int = 64, seed: int = 12345, must_include=
         if int(i) not in forced:
             chosen.append(int(i))
     return np.asarray(sorted(chosen[:max(n, len(forced))]), dtype=np.int32)
+
+
+class Drift:
+    """Per-step drift of a multi-layer config's Q/K/V on the device (the reuse-loop input).
+
+    X_s = X_{s-1} + amount * rms(X_0[layer, head]) * eps_s, eps_s ~ N(0, 1) drawn fresh for every step, layer and tensor
+    from a torch generator seeded with (seed, step, layer); rms over the real rows of each head of the step-0 tensor.
+    The walk is kept in fp32 master copies; `tokens(layer)` returns the rounded tensors the kernels read (bf16 by
+    round-to-nearest-even, the same rounding as the host generator).
+    """
+
+    def __init__(self, cfg: "LayerConfig", layers: list, device="cuda", amount: float | None = None, seed: int = 0):
+        import torch
+        self.torch = torch
+        self.cfg = cfg
+        self.device = device
+        self.amount = cfg.extra.get("drift", 0.02) if amount is None else amount
+        self.seed = seed
+        self.step = 0
+        self.master = []   # per layer: (q, k, v) fp32 [H][Np][d]
+        self.rms = []      # per layer: (3, H) fp32
+        n = cfg.n_tokens
+        for layer in layers:
+            ts = tuple(torch.from_numpy(layer.all_f32(name)).to(device) for name in ("q", "k", "v"))
+            self.master.append(ts)
+            self.rms.append(torch.stack([t[:, :n].pow(2).mean(dim=(1, 2)).sqrt() for t in ts]))
+
+    def advance(self):
+        """Apply one drift step to every layer."""
+        torch = self.torch
+        self.step += 1
+        n = self.cfg.n_tokens
+        for li, ts in enumerate(self.master):
+            g = torch.Generator(device=self.device)
+            g.manual_seed((self.seed * 1_000_003 + self.step) * 4099 + li)
+            for ti, t in enumerate(ts):
+                eps = torch.randn(t[:, :n].shape, generator=g, device=self.device, dtype=torch.float32)
+                t[:, :n].add_(eps * (self.amount * self.rms[li][ti]).view(-1, 1, 1))
+
+    def tokens(self, li: int):
+        """The current rounded q, k, v of layer li as device tensors of the config dtype."""
+        torch = self.torch
+        dt = torch.bfloat16 if self.cfg.dtype == "bf16" else torch.float32
+        return tuple(t.to(dt) for t in self.master[li])
