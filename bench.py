@@ -335,6 +335,27 @@ def run_native(args, cfg):
                "unit": "TFLOP/s (dense-equivalent, sparse attention incl. host copies)",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_call": round(t_e2e / K * 1e3, 3)}
 
+    # Outside the timed region: block density at each tau, and the fixed-count top-k ablation at matched mean
+    # coverage (the LoSA page's "retained mass vs. a fixed sparsity ratio"), both on this step's exact masses.
+    rows = cfg.heads * cfg.n_blocks
+    density = {}
+    for tau in (0.9, 0.95, 0.99, 1.0):
+        buf.select(tau)
+        density[str(tau)] = round(int(buf.indptr[-1].item()) / (rows * cfg.n_blocks), 6)
+    m = buf.mass.cpu().numpy().reshape(rows, cfg.n_blocks).astype(np.float64)
+    buf.select(args.tau)
+    gi, gk, _ = buf.csr_host()
+    k_match = max(1, int(round(len(gk) / rows)))
+    row_tau = np.array([m[r, gk[gi[r]:gi[r + 1]]].sum() for r in range(rows)]) / m.sum(axis=1)
+    buf.select_topk(k_match)
+    ti, tk, _ = buf.csr_host()
+    row_topk = np.array([m[r, tk[ti[r]:ti[r + 1]]].sum() for r in range(rows)]) / m.sum(axis=1)
+    buf.select(args.tau)
+    ablation = {"k_blocks_matched": k_match, "recall_mass_rule": round(float(row_tau.mean()), 6),
+                "recall_topk": round(float(row_topk.mean()), 6),
+                "worst_row_recall_mass_rule": round(float(row_tau.min()), 6),
+                "worst_row_recall_topk": round(float(row_topk.min()), 6)}
+
     pk = peaks()
     per_sparse = t_sparse / K
     per_prof = t_prof / K
@@ -365,6 +386,8 @@ def run_native(args, cfg):
         "dense_equiv_tflops": round(K * work["dense_equiv_flop"] / t_sparse / 1e12, 3),
         "kept_block_tflops": round(work["sparse_flop"] / per_sparse / 1e12, 3),
         "block_density": round(nnz / (cfg.heads * cfg.n_blocks ** 2), 5),
+        "block_density_by_tau": density,
+        "topk_ablation": ablation,
         "nnz_blocks": nnz,
         "roofline": roof[dominant],
         "rooflines": roof,
@@ -388,6 +411,28 @@ def run_native(args, cfg):
 
 # ------------------------------------------------------------------------------------------ reuse loop
 
+def dense_reference_fp64(cfg, q, k, v, scale, items):
+    """Dense attention of the listed items in float64 with plain torch CPU ops, for the loop's reported
+    approximation error (rows t >= N are NaN)."""
+    import torch
+    R, nq, N = cfg.block, cfg.n_blocks, cfg.n_tokens
+    out = np.full((len(items), R, cfg.head_dim), np.nan)
+    kf, vf = k.double().cpu(), v.double().cpu()
+    qf = q.double().cpu()
+    for t, it in enumerate(items):
+        h, i = divmod(int(it), nq)
+        rows = min(R, N - i * R)
+        s = (qf[h, i * R:i * R + rows] @ kf[h, :N].T) * scale
+        out[t, :rows] = (torch.softmax(s, dim=-1) @ vf[h, :N]).numpy()
+    return out
+
+
+def pattern_recall(mass, indptr, kv_idx):
+    """Recall of a CSR pattern under masses [rows][nk]: retained mass over total mass."""
+    kept = sum(float(mass[r, kv_idx[indptr[r]:indptr[r + 1]]].sum()) for r in range(mass.shape[0]))
+    return kept / float(mass.sum())
+
+
 def run_loop(args, cfg):
     """Denoising-loop reuse at the Wan2.1-480p shape: steps before the construction step t0 are dense, step t0
     profiles every layer and selects its pattern (t0 = 0 by default; the LoSA page's setup uses t0 = 3), later steps
@@ -399,7 +444,6 @@ def run_loop(args, cfg):
     import free_block_sparse_losa_b200 as L
     from free_block_sparse_losa_b200.harness import LayerBuffers
     from losa_synth import Drift
-    import oracle
 
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -453,8 +497,7 @@ def run_loop(args, cfg):
                 step_dense.append((e1, e2))
                 if step in report_steps and li == 0:
                     torch.cuda.synchronize()
-                    qf, kf, vf = (x.float().cpu().numpy() for x in (q, k, v))
-                    ref, _ = oracle.dense(qf, kf, vf, cfg.n_tokens, cfg.block, scale, items)
+                    ref = dense_reference_fp64(cfg, q, k, v, scale, items)
                     got = b.o.float().cpu().numpy().reshape(cfg.heads * cfg.n_blocks, cfg.block, cfg.head_dim)
                     gd = dense_o.float().cpu().numpy().reshape(got.shape)
                     ok = ~np.isnan(ref)
@@ -465,7 +508,7 @@ def run_loop(args, cfg):
                     probe.profile(q, k, v, scale)
                     m = probe.mass.cpu().numpy().reshape(probe.rows, probe.nk).astype(np.float64)
                     gi, gk, _ = b.csr_host()
-                    recall[step] = oracle.recall(m, gi, gk)
+                    recall[step] = pattern_recall(m, gi, gk)
             torch.cuda.synchronize()
             t_sparse_path.append(sum(a.elapsed_time(z) for a, z in step_sparse))
             t_dense_path.append(sum(a.elapsed_time(z) for a, z in step_dense))

@@ -11,7 +11,7 @@ import ctypes
 import os
 
 __all__ = ["LosaShape", "LosaError", "make_shape", "losa_dense_profile", "losa_select", "losa_select_noalloc",
-           "losa_sparse_attn",
+           "losa_select_topk", "losa_sparse_attn",
            "losa_select_workspace_bytes", "losa_get_device_error", "losa_selftest_wait_timeout",
            "losa_set_wait_limit_ns", "losa_status_string", "losa_version", "library_path", "load",
            "DTYPE_F32", "DTYPE_BF16", "STATUS"]
@@ -62,6 +62,7 @@ def load():
     L.losa_dense_profile.argtypes = [sp, vp, vp, vp, f32, vp, vp, vp, vp]
     L.losa_select.argtypes = [sp, vp, f64, vp, vp, i64, vp, vp, sz, vp]
     L.losa_select_noalloc.argtypes = [sp, vp, f64, vp, vp, i64, vp, vp]
+    L.losa_select_topk.argtypes = [sp, vp, i32, vp, vp, i64, vp, vp, sz, vp]
     L.losa_select_workspace_bytes.argtypes = [sp]
     L.losa_select_workspace_bytes.restype = sz
     L.losa_sparse_attn.argtypes = [sp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp]
@@ -72,7 +73,8 @@ def load():
     L.losa_status_string.argtypes = [i32]
     L.losa_status_string.restype = ctypes.c_char_p
     L.losa_version.restype = ctypes.c_int
-    for name in ("losa_dense_profile", "losa_select", "losa_select_noalloc", "losa_sparse_attn", "losa_get_device_error",
+    for name in ("losa_dense_profile", "losa_select", "losa_select_noalloc", "losa_select_topk", "losa_sparse_attn",
+                 "losa_get_device_error",
                  "losa_selftest_wait_timeout"):
         getattr(L, name).restype = i32
     _lib = L
@@ -123,6 +125,15 @@ def losa_select(shape, mass, tau, indptr, kv_block_idx, order, workspace, idx_ca
     st = load().losa_select(ctypes.byref(shape), _ptr(mass), float(tau), _ptr(indptr), _ptr(kv_block_idx), int(cap),
                             _ptr(order), _ptr(workspace), int(wsb), _stream(stream))
     return _check(st, "losa_select", raise_on_error)
+
+
+def losa_select_topk(shape, mass, k_blocks, indptr, kv_block_idx, order, workspace, idx_capacity=None, ws_bytes=None,
+                     stream=None, raise_on_error=True):
+    cap = kv_block_idx.numel() if idx_capacity is None else idx_capacity
+    wsb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    st = load().losa_select_topk(ctypes.byref(shape), _ptr(mass), int(k_blocks), _ptr(indptr), _ptr(kv_block_idx),
+                                 int(cap), _ptr(order), _ptr(workspace), int(wsb), _stream(stream))
+    return _check(st, "losa_select_topk", raise_on_error)
 
 
 def losa_select_noalloc(shape, mass, tau, indptr, kv_block_idx, order, idx_capacity=None, stream=None,

@@ -270,7 +270,7 @@ losa_status losa_select(const losa_shape* shape, const float* mass, double tau, 
     if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem1) != cudaSuccess)
         return LOSA_ERR_CUDA;
-    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, counts,
+    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, 0, counts,
                                                                                          staged);
     if ((st = launch_status()) != LOSA_OK) return st;
 
@@ -282,6 +282,44 @@ losa_status losa_select(const losa_shape* shape, const float* mass, double tau, 
     select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
     if ((st = launch_status()) != LOSA_OK) return st;
 
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
+    return launch_status();
+}
+
+losa_status losa_select_topk(const losa_shape* shape, const float* mass, int32_t k_blocks, int32_t* indptr,
+                             int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (k_blocks < 1) return LOSA_ERR_INVALID_ARG;
+    if (!aligned16(mass) || !indptr || !kv_block_idx || !order || !aligned16(workspace)) return LOSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
+         reinterpret_cast<uintptr_t>(order)) & 3u)
+        return LOSA_ERR_INVALID_ARG;
+    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
+    const long long rows = (long long)shape->heads * nq;
+    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
+    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
+    if (ws_bytes < select_ws_bytes(shape)) return LOSA_ERR_CAPACITY;
+    int32_t* staged = static_cast<int32_t*>(workspace);
+    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
+    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
+    const int n2 = next_pow2(nk);
+    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
+    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem1) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, 1.0, k_blocks,
+                                                                                         counts, staged);
+    if ((st = launch_status()) != LOSA_OK) return st;
+    const int r2 = next_pow2((int)rows);
+    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
+    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem2) != cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
+    if ((st = launch_status()) != LOSA_OK) return st;
     const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
     select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
     return launch_status();
@@ -402,7 +440,7 @@ extern "C" losa_status losa_select_noalloc(const losa_shape* shape, const float*
     if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem1) != cudaSuccess)
         return LOSA_ERR_CUDA;
-    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, counts,
+    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, 0, counts,
                                                                                          staged);
     if ((st = launch_status()) != LOSA_OK) return st;
     const int r2 = next_pow2((int)rows);

@@ -1,4 +1,6 @@
-// Mass-threshold block selection (LoSA page, Methodology Summary, "One-time pattern construction").
+// Mass-threshold block selection (LoSA page, Methodology Summary, "One-time pattern construction"), and the
+// fixed-count top-k rule the page's ablation compares it with (Experiments Summary, "Retained mass vs. a fixed
+// sparsity ratio").
 //
 // Three launches, all stream-ordered:
 //   1. select_rows_kernel    one CTA per (head, query block) row: bitonic sort of the row's masses in shared memory
@@ -66,9 +68,10 @@ __device__ __forceinline__ void bitonic_sort_smem(K* keys, int n) {
 }
 
 // Kernel 1. Dynamic shared memory: n2 uint64 keys + nk bytes of kept flags (n2 = next power of two >= nk).
+// topk > 0 switches from the mass threshold to a fixed count: keep the topk largest blocks (ties by index).
 template <int NT>
 __global__ void __launch_bounds__(NT) select_rows_kernel(const float* __restrict__ mass, int nk, int n2, double tau,
-                                                          int32_t* __restrict__ counts,
+                                                          int topk, int32_t* __restrict__ counts,
                                                           int32_t* __restrict__ staged) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint64_t* keys = reinterpret_cast<uint64_t*>(smem_raw);
@@ -130,7 +133,8 @@ __global__ void __launch_bounds__(NT) select_rows_kernel(const float* __restrict
     }
     uint64_t n_below;
     block_excl_scan_u64<NT>(below, warp_tot, n_below);
-    const int s = (n_below + 1 < (uint64_t)nk) ? (int)(n_below + 1) : nk;
+    int s = (n_below + 1 < (uint64_t)nk) ? (int)(n_below + 1) : nk;
+    if (topk > 0) s = topk < nk ? topk : nk;
 
     for (int p = threadIdx.x; p < s; p += NT) kept[(uint32_t)(keys[p] & 0xffffffffu)] = 1;
     __syncthreads();

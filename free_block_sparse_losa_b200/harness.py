@@ -8,7 +8,7 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from . import (DTYPE_BF16, DTYPE_F32, losa_dense_profile, losa_select, losa_select_workspace_bytes,
+from . import (DTYPE_BF16, DTYPE_F32, losa_dense_profile, losa_select, losa_select_topk, losa_select_workspace_bytes,
                losa_sparse_attn, make_shape)
 
 
@@ -63,6 +63,10 @@ class LayerBuffers:
     def select(self, tau, mass=None, stream=None):
         losa_select(self.shape, self.mass if mass is None else mass, tau, self.indptr, self.kv_idx, self.order,
                     self.workspace, stream=stream)
+
+    def select_topk(self, k_blocks, mass=None, stream=None):
+        losa_select_topk(self.shape, self.mass if mass is None else mass, k_blocks, self.indptr, self.kv_idx,
+                         self.order, self.workspace, stream=stream)
 
     def sparse(self, q, k, v, scale, out=None, lse=None, stream=None, order=True):
         losa_sparse_attn(self.shape, q, k, v, scale, self.indptr, self.kv_idx, self.order if order else None,

@@ -17,6 +17,9 @@
  *     (a multiple of the block sizes, N <= Np < N + block). Keys t >= N take no part in any softmax; output
  *     rows t >= N are written but carry no meaning. Base pointers must be 16-byte aligned.
  *   - An "item" is one (head, query block) pair with id h * nq + i, nq = Np / block_q, nk = Np / block_k.
+ *   - A batch (several samples, or the conditional and unconditional branches of classifier-free guidance) is passed
+ *     as heads = B * H with tensors [B][H][Np][d]: every (sample or branch, head) gets its own pattern, as the LoSA
+ *     page's Methodology Summary keeps separate patterns for the two guidance branches.
  *   - Status codes below; LOSA_ERR_CUDA covers launch failures reported by the CUDA runtime.
  *
  * Supported shapes: dtype BF16 with head_dim 128 and block_q = block_k = 128 (tensor-core path), or dtype F32
@@ -94,6 +97,16 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
 losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
                         int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
                         size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Fixed-count selection, the ablation baseline of the LoSA page (Experiments Summary, "Retained mass vs. a fixed
+ * sparsity ratio": keep the same number of blocks in every row, matched to the mass rule's mean coverage).
+ * Same arguments, outputs and ordering as losa_select, with k_blocks (>= 1; rows keep min(k_blocks, nk)) in place of
+ * tau: each row keeps its k_blocks largest-mass blocks (ties to the lower index), listed in ascending order.
+ */
+losa_status losa_select_topk(const losa_shape* shape, const float* mass, int32_t k_blocks, int32_t* indptr,
+                             int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream);
 
 /* Bytes of device workspace losa_select needs for this shape (0 if the shape is invalid). */
 size_t losa_select_workspace_bytes(const losa_shape* shape);

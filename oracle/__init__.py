@@ -37,11 +37,12 @@ def lib():
         L.oracle_mass.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, i32, vp, vp]
         L.oracle_select_f32.argtypes = [i32, i32, vp, f64, vp, vp]
         L.oracle_select_f64.argtypes = [i32, i32, vp, f64, vp, vp]
+        L.oracle_select_topk.argtypes = [i32, i32, vp, i32, vp, vp]
         L.oracle_lpt_order.argtypes = [i32, vp, vp]
         L.oracle_sparse.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, vp, vp, vp, i32, vp, vp, vp]
         L.oracle_recall.argtypes = [i32, i32, vp, vp, vp, vp]
         L.oracle_recall.restype = f64
-        for name in ("oracle_dense", "oracle_mass", "oracle_select_f32", "oracle_select_f64",
+        for name in ("oracle_dense", "oracle_mass", "oracle_select_f32", "oracle_select_f64", "oracle_select_topk",
                      "oracle_lpt_order", "oracle_sparse"):
             getattr(L, name).restype = i32
         _lib = L
@@ -111,6 +112,16 @@ def select(m, tau: float):
         m = np.ascontiguousarray(m, dtype=np.float64)
         rc = lib().oracle_select_f64(nk, rows, _p(m), tau, _p(counts), _p(idx))
     _check(rc, "oracle_select")
+    return counts, idx
+
+
+def select_topk(m, k: int):
+    """Fixed-count selection on fp32 masses [rows][nk]: (counts, idx) as select()."""
+    m = np.ascontiguousarray(m, dtype=np.float32)
+    rows, nk = m.shape
+    counts = np.empty(rows, dtype=np.int32)
+    idx = np.full((rows, nk), -1, dtype=np.int32)
+    _check(lib().oracle_select_topk(nk, rows, _p(m), int(k), _p(counts), _p(idx)), "oracle_select_topk")
     return counts, idx
 
 

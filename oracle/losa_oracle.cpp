@@ -207,6 +207,25 @@ int oracle_select_f64(int nk, int n_rows, const double* mass, double tau, int32_
     return bad ? -1 : 0;
 }
 
+// Fixed-count selection (the LoSA page's ablation baseline, Experiments Summary, "Retained mass vs. a fixed sparsity
+// ratio"): each row keeps its k largest-mass blocks, ties to the lower index (R3), listed ascending (R5).
+int oracle_select_topk(int nk, int n_rows, const float* mass, int k, int32_t* counts, int32_t* idx) {
+    if (nk <= 0 || n_rows < 0 || k < 1) return -1;
+    const int s = std::min(k, nk);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int r = 0; r < n_rows; ++r) {
+        const float* m = mass + (size_t)r * nk;
+        std::vector<int> ord(nk);
+        std::iota(ord.begin(), ord.end(), 0);
+        std::sort(ord.begin(), ord.end(), [&](int a, int b) { return m[a] > m[b] || (m[a] == m[b] && a < b); });
+        std::vector<int> kept(ord.begin(), ord.begin() + s);
+        std::sort(kept.begin(), kept.end());
+        for (int t = 0; t < s; ++t) idx[(size_t)r * nk + t] = kept[t];
+        counts[r] = s;
+    }
+    return 0;
+}
+
 // Longest-first work order (R6): item ids sorted by count descending, ties by ascending id.
 int oracle_lpt_order(int n, const int32_t* counts, int32_t* order) {
     if (n < 0) return -1;

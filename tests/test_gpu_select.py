@@ -76,6 +76,27 @@ def test_select_full_size_hunyuan_rows(oracle_mod):
     _run((H, nb, nb, 128, 128), m, 0.99, oracle_mod)
 
 
+@pytest.mark.parametrize("H,nb,k", [(1, 1, 1), (2, 31, 4), (4, 256, 12), (1, 929, 40), (2, 64, 64), (2, 64, 100)])
+def test_select_topk_matches_oracle(H, nb, k, oracle_mod):
+    rng = np.random.default_rng(H * 7 + nb)
+    m = _masses(rng, H * nb, nb, "peaked" if nb > 4 else "ties")
+    shape = L.make_shape(H, nb * 128 - 1, nb * 128, 128, 128, 128, "bf16")
+    rows = H * nb
+    dev = torch.from_numpy(m.ravel()).cuda()
+    indptr = torch.empty(rows + 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(rows * nb, dtype=torch.int32, device="cuda")
+    order = torch.empty(rows, dtype=torch.int32, device="cuda")
+    ws = torch.empty(L.losa_select_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    L.losa_select_topk(shape, dev, k, indptr, idx, order, ws)
+    assert L.losa_get_device_error() == 0
+    counts, ref = oracle_mod.select_topk(m, k)
+    ri, rk = oracle_mod.to_csr(counts, ref)
+    gi = indptr.cpu().numpy()
+    np.testing.assert_array_equal(gi, ri)
+    np.testing.assert_array_equal(idx.cpu().numpy()[:gi[-1]], rk)
+    np.testing.assert_array_equal(order.cpu().numpy(), oracle_mod.lpt_order(counts))
+
+
 def test_select_reports_bad_mass():
     shape = L.make_shape(1, 1023, 1024, 128, 128, 128, "bf16")
     rows, nk = 8, 8

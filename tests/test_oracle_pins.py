@@ -302,6 +302,23 @@ def test_select_brute_force_tiny():
             assert len(winners) == 1 and list(winners[0]) == kept
 
 
+def test_select_topk_keeps_k_largest_with_index_ties():
+    """Brute force: the kept set is the k largest masses, ties resolved toward lower indices; equal masses keep
+    the first k indices; k >= nk keeps everything."""
+    rng = np.random.default_rng(21)
+    import oracle
+    for trial in range(60):
+        nk = int(rng.integers(1, 40))
+        m = rng.integers(0, 6, nk).astype(np.float32) if trial % 2 else rng.random(nk).astype(np.float32)
+        k = int(rng.integers(1, nk + 3))
+        counts, idx = oracle.select_topk(m[None], k)
+        kept = list(idx[0, :counts[0]])
+        want = sorted(sorted(range(nk), key=lambda j: (-float(m[j]), j))[:min(k, nk)])
+        assert kept == want
+    counts, idx = oracle.select_topk(np.full((1, 8), 0.125, np.float32), 3)
+    assert list(idx[0, :counts[0]]) == [0, 1, 2]
+
+
 def test_select_rejects_bad_tau():
     import oracle
     m = np.full((1, 4), 0.25)
