@@ -34,7 +34,7 @@ from losa_synth import CONFIGS, make_layer, sample_items  # noqa: E402
 
 WORKLOADS = {"hunyuan720": 3, "wan14b720": 2, "wan1.3b480": 1, "tiny": 0, "loop": 4}
 METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select ms"
-KERNELS_PER_STEP = {"dense_profile": 2, "select": 3, "sparse_attn": 1}
+KERNELS_PER_STEP = {"dense_profile": 1, "select": 3, "sparse_attn": 1}
 
 
 def peaks():
@@ -120,6 +120,28 @@ class ClockSampler:
         loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def kernel_source_hash():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "free_block_sparse_losa_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload_name):
+    """Per-launch DRAM bytes from the committed ncu summary, only if the kernels are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic_hunyuan720.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        t = json.load(f)
+    if t.get("workload") != workload_name or t.get("source_hash") != kernel_source_hash():
+        return {}
+    return t
 
 
 def roofline(name, bound, work, seconds, pk, unit, traffic=None, peak_kind="sustained"):
@@ -360,13 +382,14 @@ def run_native(args, cfg):
     per_sparse = t_sparse / K
     per_prof = t_prof / K
     per_sel = t_sel / K
+    tr = measured_traffic(cfg.name)
     roof = {
-        "dense_profile": roofline("attn_tc_kernel<Fwd> + attn_tc_kernel<Mass> (losa_dense_profile)", "tensor",
-                                  work["profile_flop"], per_prof, pk, "TFLOP/s"),
+        "dense_profile": roofline("attn_tc_kernel<1> (losa_dense_profile: dense forward + block masses)", "tensor",
+                                  work["profile_flop"], per_prof, pk, "TFLOP/s", tr.get("dense_profile")),
         "select": roofline("select_rows + select_finalize + select_scatter (losa_select)", "hbm",
-                           work["select_bytes"], per_sel, pk, "GB/s"),
-        "sparse_attn": roofline("attn_tc_kernel<Fwd> over retained lists (losa_sparse_attn)", "tensor",
-                                work["sparse_flop"], per_sparse, pk, "TFLOP/s"),
+                           work["select_bytes"], per_sel, pk, "GB/s", tr.get("select")),
+        "sparse_attn": roofline("attn_tc_kernel<0> over the retained lists (losa_sparse_attn)", "tensor",
+                                work["sparse_flop"], per_sparse, pk, "TFLOP/s", tr.get("sparse_attn")),
     }
     dominant = max(("dense_profile", per_prof), ("select", per_sel), ("sparse_attn", per_sparse),
                    key=lambda x: x[1])[0]
