@@ -191,6 +191,28 @@ int next_pow2(int n) {
     return p;
 }
 
+// Kernel 1 of the selection: the warp-per-row register form for nk <= 1024, else the CTA shared-memory form.
+losa_status launch_select_rows(const float* mass, int nk, int rows, double tau, int topk, int32_t* counts,
+                               int32_t* staged, cudaStream_t stream) {
+    const unsigned wgrid = (unsigned)((rows + 7) / 8);
+    if (nk <= 32) select_rows_warp_kernel<1><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else if (nk <= 64) select_rows_warp_kernel<2><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else if (nk <= 128) select_rows_warp_kernel<4><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else if (nk <= 256) select_rows_warp_kernel<8><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else if (nk <= 512) select_rows_warp_kernel<16><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else if (nk <= 1024) select_rows_warp_kernel<32><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+    else {
+        const int n2 = next_pow2(nk);
+        const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
+        if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem1) != cudaSuccess)
+            return LOSA_ERR_CUDA;
+        select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, topk,
+                                                                                             counts, staged);
+    }
+    return launch_status();
+}
+
 size_t select_ws_bytes(const losa_shape* s) {
     const size_t rows = (size_t)s->heads * (s->n_padded / s->block_q);
     const size_t nk = (size_t)(s->n_padded / s->block_k);
@@ -265,14 +287,7 @@ losa_status losa_select(const losa_shape* shape, const float* mass, double tau, 
     const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
     int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
 
-    const int n2 = next_pow2(nk);
-    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
-    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem1) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, 0, counts,
-                                                                                         staged);
-    if ((st = launch_status()) != LOSA_OK) return st;
+    if ((st = launch_select_rows(mass, nk, (int)rows, tau, 0, counts, staged, stream)) != LOSA_OK) return st;
 
     const int r2 = next_pow2((int)rows);
     const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
@@ -305,14 +320,7 @@ losa_status losa_select_topk(const losa_shape* shape, const float* mass, int32_t
     int32_t* staged = static_cast<int32_t*>(workspace);
     const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
     int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
-    const int n2 = next_pow2(nk);
-    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
-    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem1) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, 1.0, k_blocks,
-                                                                                         counts, staged);
-    if ((st = launch_status()) != LOSA_OK) return st;
+    if ((st = launch_select_rows(mass, nk, (int)rows, 1.0, k_blocks, counts, staged, stream)) != LOSA_OK) return st;
     const int r2 = next_pow2((int)rows);
     const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
     if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -435,14 +443,7 @@ extern "C" losa_status losa_select_noalloc(const losa_shape* shape, const float*
     const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
     int32_t* counts = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(scratch) + staged_bytes);
 
-    const int n2 = next_pow2(nk);
-    const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
-    if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem1) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_rows_kernel<kSelectThreads><<<(unsigned)rows, kSelectThreads, smem1, stream>>>(mass, nk, n2, tau, 0, counts,
-                                                                                         staged);
-    if ((st = launch_status()) != LOSA_OK) return st;
+    if ((st = launch_select_rows(mass, nk, (int)rows, tau, 0, counts, staged, stream)) != LOSA_OK) return st;
     const int r2 = next_pow2((int)rows);
     const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
     if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -157,6 +157,125 @@ __global__ void __launch_bounds__(NT) select_rows_kernel(const float* __restrict
     if (threadIdx.x == 0) counts[row] = s;
 }
 
+// Kernel 1, warp-per-row form for rows of nk <= 32 * E keys (E a power of two <= 32): the same bitonic network held
+// in registers. Lane l owns sorted positions [l*E, l*E + E): compare-exchange partners at distance j < E sit in the
+// same lane, partners at distance j >= E in lane l ^ (j / E) (exchanged by shuffle). No shared memory or block
+// barrier is involved in the sort; the integer prefix is an in-lane scan plus a warp scan of lane totals; the kept
+// set is turned into ascending block order through a per-warp bitmap of E words.
+template <int E>
+__global__ void __launch_bounds__(256) select_rows_warp_kernel(const float* __restrict__ mass, int nk, int rows,
+                                                                double tau, int topk, int32_t* __restrict__ counts,
+                                                                int32_t* __restrict__ staged) {
+    __shared__ uint32_t bitmap_all[8][32];
+    const int warp = threadIdx.x >> 5;
+    const int lane = (int)lane_id();
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    uint32_t* bitmap = bitmap_all[warp];
+    const float* m = mass + (size_t)row * nk;
+    uint64_t key[E];
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = lane * E + e;
+        uint64_t kk = ~0ull;
+        if (j < nk) {
+            float xv = m[j];
+            if (!(xv >= 0.0f) || isinf(xv)) {
+                bad = true;
+                xv = 0.0f;
+            }
+            const uint32_t bits = (xv == 0.0f) ? 0u : __float_as_uint(xv);
+            kk = ((uint64_t)(~bits) << 32) | (uint32_t)j;
+        }
+        key[e] = kk;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_device_error, kDevErrBadData);
+    // Bitonic sort, ascending, of the 32 * E keys.
+#pragma unroll
+    for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j < E) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int pe = e ^ j;
+                    if (pe > e) {
+                        const int i = lane * E + e;
+                        const bool up = (i & k) == 0;
+                        const uint64_t a = key[e], b = key[pe];
+                        const bool swap = (a > b) == up;
+                        key[e] = swap ? b : a;
+                        key[pe] = swap ? a : b;
+                    }
+                }
+            } else {
+                const int dl = j / E;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const uint64_t other = __shfl_xor_sync(0xffffffffu, key[e], dl);
+                    const int i = lane * E + e;
+                    const bool up = (i & k) == 0;
+                    const bool lower = (lane & dl) == 0;   // this position is the lower index of the pair
+                    const uint64_t mn = key[e] < other ? key[e] : other;
+                    const uint64_t mx = key[e] < other ? other : key[e];
+                    key[e] = (lower == up) ? mn : mx;
+                }
+            }
+        }
+    }
+    // Integer prefix over sorted positions; u = ceil(M * 2^52) exactly in fp64.
+    uint64_t local = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        local += (uint64_t)ceil((double)__uint_as_float(~(uint32_t)(key[e] >> 32)) * 4503599627370496.0);
+    const uint64_t incl = warp_incl_scan_u64(local);
+    const uint64_t total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint64_t target = (uint64_t)ceil(__dmul_rn(tau, __ull2double_rn(total)));
+    uint64_t run = incl - local;
+    int below = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        run += (uint64_t)ceil((double)__uint_as_float(~(uint32_t)(key[e] >> 32)) * 4503599627370496.0);
+        below += (run < target) ? 1 : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+    int s = (below + 1 < nk) ? below + 1 : nk;
+    if (topk > 0) s = topk < nk ? topk : nk;
+    // Kept set (sorted positions < s) -> bitmap by block index -> ascending compaction.
+    for (int w = lane; w < E; w += 32) bitmap[w] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (lane * E + e < s) {
+            const uint32_t j = (uint32_t)(key[e] & 0xffffffffu);
+            atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+        }
+    __syncwarp();
+    // Lane l emits block indices [l*E, l*E + E) that are kept, at its exclusive prefix of kept counts.
+    uint32_t myb = 0;
+    const int j0 = lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = j0 + e;
+        if (j < nk && ((bitmap[j >> 5] >> (j & 31)) & 1u)) myb |= 1u << e;
+    }
+    const int cnt = __popc(myb);
+    int pre = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+    }
+    pre -= cnt;
+    int32_t* out = staged + (size_t)row * nk;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if ((myb >> e) & 1u) out[pre++] = j0 + e;
+    if (lane == 0) counts[row] = s;
+}
+
 // Kernel 2 (one CTA, NT threads). Dynamic shared memory: n2 uint32 keys (n2 = power of two >= rows).
 template <int NT>
 __global__ void __launch_bounds__(NT) select_finalize_kernel(const int32_t* __restrict__ counts, int rows, int nk,
