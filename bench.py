@@ -53,14 +53,14 @@ def work_model(cfg, nnz):
     """Algorithmic work per call. Tensor FLOPs count 2 per multiply-add; the dense-equivalent figure uses the
     real token count N, kept-block figures count whole 128 x 128 tiles."""
     H, N, Np, d, B = cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block
-    nq = Np // B
+    nq, nkb, C = Np // B, Np // cfg.kblock, cfg.kblock
     return {
         "dense_equiv_flop": 4.0 * H * N * N * d,
         "profile_flop": 6.0 * H * N * N * d,          # Q K^T + P V forward, then Q K^T again for the masses
         "profile_exp": 2.0 * H * N * N,
-        "sparse_flop": 4.0 * B * B * d * nnz,         # kept tiles only
-        "sparse_exp": float(B * B * nnz),
-        "select_bytes": 4.0 * H * nq * nq + 4.0 * (nnz + 2 * H * nq + 1),  # read M, write CSR + order
+        "sparse_flop": 4.0 * B * C * d * nnz,         # kept blocks only (R x C each)
+        "sparse_exp": float(B * C * nnz),
+        "select_bytes": 4.0 * H * nq * nkb + 4.0 * (nnz + 2 * H * nq + 1),  # read M, write CSR + order
     }
 
 
@@ -363,8 +363,8 @@ def run_native(args, cfg):
     density = {}
     for tau in (0.9, 0.95, 0.99, 1.0):
         buf.select(tau)
-        density[str(tau)] = round(int(buf.indptr[-1].item()) / (rows * cfg.n_blocks), 6)
-    m = buf.mass.cpu().numpy().reshape(rows, cfg.n_blocks).astype(np.float64)
+        density[str(tau)] = round(int(buf.indptr[-1].item()) / (rows * cfg.n_kblocks), 6)
+    m = buf.mass.cpu().numpy().reshape(rows, cfg.n_kblocks).astype(np.float64)
     buf.select(args.tau)
     gi, gk, _ = buf.csr_host()
     k_match = max(1, int(round(len(gk) / rows)))
@@ -399,7 +399,7 @@ def run_native(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
         "data": "synthetic (seeded grid-structured Q/K/V, see DESIGN.md)",
         "config": {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens, "n_padded": cfg.n_padded,
-                   "head_dim": cfg.head_dim, "block": cfg.block, "tau": args.tau,
+                   "head_dim": cfg.head_dim, "block": cfg.block, "block_k": cfg.kblock, "tau": args.tau,
                    "l2": "inputs larger than L2 (3 x %.0f MB of Q/K/V per layer)" % (q.numel() * 2 / 1e6),
                    "parallelism": f"replicas x{world} (one independent layer per GPU)"},
         "sparse_attn_ms": round(per_sparse * 1e3, 3),
@@ -408,7 +408,7 @@ def run_native(args, cfg):
         "profile_select_ms": round((per_prof + per_sel) * 1e3, 3),
         "dense_equiv_tflops": round(K * work["dense_equiv_flop"] / t_sparse / 1e12, 3),
         "kept_block_tflops": round(work["sparse_flop"] / per_sparse / 1e12, 3),
-        "block_density": round(nnz / (cfg.heads * cfg.n_blocks ** 2), 5),
+        "block_density": round(nnz / (cfg.heads * cfg.n_blocks * cfg.n_kblocks), 5),
         "block_density_by_tau": density,
         "topk_ablation": ablation,
         "nnz_blocks": nnz,
@@ -569,6 +569,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="hunyuan720")
     ap.add_argument("--tau", type=float, default=0.99)
+    ap.add_argument("--block-k", type=int, default=0, choices=[0, 32, 128],
+                    help="key block size C (0: the workload's, 128; 32 is the LoSA page's setup)")
     ap.add_argument("--cpu-items", type=int, default=0, help="oracle sample size (0: one item per host thread)")
     ap.add_argument("--ref-items", type=int, default=0, help="reference-arm items per step (0: half the threads)")
     ap.add_argument("--loop-layers", type=int, default=0, help="reuse loop: layers (0: the config's 30)")
@@ -579,6 +581,9 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     cfg = CONFIGS[WORKLOADS[args.workload]]
+    if args.block_k:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, block_k=args.block_k)
     if args.workload == "loop":
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the reuse loop has no CPU-oracle arm; its "

@@ -51,7 +51,8 @@ constexpr uint32_t tc_smem_bytes() {
 }
 
 struct TcArgs {
-    int H, N, Np, nq, nk, n_items;
+    int H, N, Np, nq, nk, n_items;  // nk: 128-key tiles per head (Np / 128)
+    int nkb;                        // key blocks of the selection (Np / C): nk for C = 128, 4 * nk for C = 32
     float scale_log2;              // logit scale times log2(e)
     const int32_t* indptr;         // null: dense list 0..nk-1
     const int32_t* kv_idx;
@@ -82,7 +83,9 @@ __device__ __forceinline__ bool wait_bounded_warp(uint32_t bar, uint32_t parity,
 }
 
 struct ItemInfo {
-    int id, h, qb, begin, count;
+    int id, h, qb, begin;
+    int count;  // list entries (key blocks); every block for a dense call
+    int tiles;  // forward 128-key tiles: ceil(count / SUB) for a list, nk for a dense call
 };
 
 // Item of CTA round `round` (false past the end of the work order).
@@ -96,19 +99,41 @@ __device__ __forceinline__ bool item_of_round(const TcArgs& a, int round, ItemIn
     if (a.indptr) {
         it.begin = a.indptr[it.id];
         it.count = a.indptr[it.id + 1] - it.begin;
+        it.tiles = (it.count + (a.nkb / a.nk) - 1) / (a.nkb / a.nk);
     } else {
         it.begin = 0;
-        it.count = a.nk;
+        it.count = a.nkb;
+        it.tiles = a.nk;
     }
     return true;
 }
 
-// Key block of forward tile t (the producer reports out-of-range indices; everyone uses the clamped value).
-__device__ __forceinline__ int fwd_block(const TcArgs& a, const ItemInfo& it, int t) {
-    if (!a.indptr) return t;
-    const int j = a.kv_idx[it.begin + t];
-    return (j < 0) ? 0 : (j >= a.nk ? a.nk - 1 : j);
+// Block index of list entry e (clamped; the producer reports out-of-range entries).
+__device__ __forceinline__ int list_block(const TcArgs& a, const ItemInfo& it, int e) {
+    const int j = a.kv_idx[it.begin + e];
+    return (j < 0) ? 0 : (j >= a.nkb ? a.nkb - 1 : j);
 }
+
+// Real keys in each 32-key quarter of forward tile t, packed 8 bits per quarter. A quarter with no list entry (the
+// tail of a C = 32 list) has none; the ragged end of the sequence cuts the last block.
+template <int SUB>
+__device__ __forceinline__ uint32_t quarter_keys(const TcArgs& a, const ItemInfo& it, int t) {
+    uint32_t kv = 0;
+    if (SUB == 1 || !a.indptr) {
+        const int j128 = a.indptr ? list_block(a, it, t) : t;
+        const int kvalid = a.N - j128 * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) kv |= (uint32_t)min(32, max(0, kvalid - 32 * g)) << (8 * g);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int e = SUB * t + g;
+            if (e < it.count) kv |= (uint32_t)min(32, max(0, a.N - list_block(a, it, e) * 32)) << (8 * g);
+        }
+    }
+    return kv;
+}
+
 
 // 2^x on the FMA/ALU pipes, to take part of the load off the exp unit. Cody-Waite split x = n + f with n = round(x)
 // (the 1.5 * 2^23 shift leaves n in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial whose
@@ -162,13 +187,16 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 // Barrier slots of one lane (8 bytes each). Counts: P_FULL, O_FREE, S_FREE, PART take 128 arrivals, the rest 1.
 enum : uint32_t {
     L_Q_FULL = 0, L_Q_EMPTY, L_K_FULL, L_K_EMPTY, L_V_FULL, L_V_EMPTY, L_S_FULL, L_P_FULL, L_PV_DONE, L_O_FREE,
-    L_S_FREE, L_PART, L_MMA_DONE, L_COUNT
+    L_S_FREE, L_PART, L_PART2, L_MMA_DONE, L_COUNT
 };
 
-template <bool WITH_MASS>
+// SUB = key blocks per 128-key tile: 1 for C = 128, 4 for C = 32 (tmK32 / tmV32: 32-row boxes for gathering a list's
+// 32-key blocks into the quarters of a tile).
+template <bool WITH_MASS, int SUB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK32,
+                   const __grid_constant__ CUtensorMap tmV32, const TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -190,7 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x < 2) {  // thread 0 initialises lane 0's barriers, thread 1 lane 1's
         const uint32_t b0 = base + bar_off + threadIdx.x * kBarBytes;
         for (uint32_t s = 0; s < L_COUNT; ++s) {
-            const bool wide = (s == L_P_FULL || s == L_O_FREE || s == L_S_FREE || s == L_PART);
+            const bool wide = (s == L_P_FULL || s == L_O_FREE || s == L_S_FREE || s == L_PART || s == L_PART2);
             mbar_init(b0 + 8u * s, wide ? 128u : 1u);
         }
         fence_barrier_init();
@@ -203,6 +231,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        if (SUB > 1) {
+            tma_prefetch_desc(&tmK32);
+            tma_prefetch_desc(&tmV32);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -232,28 +264,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tma_load_2d_hint(sQ, &tmQ, 0, qrow, BAR(L_Q_FULL), pol_q);
                 tma_load_2d_hint(sQ + kBoxBytes, &tmQ, 64, qrow, BAR(L_Q_FULL), pol_q);
                 ++nq;
-                const int total = it.count + mass_tiles;
-                int jn = fwd_block(a, it, 0);  // block index fetched one tile ahead
+                const int total = it.tiles + mass_tiles;
                 for (int t = 0; t < total; ++t) {
-                    const bool fwd = t < it.count;
-                    const int j = jn;
-                    if (t + 1 < it.count) jn = fwd_block(a, it, t + 1);
-                    else jn = t + 1 - it.count;  // mass phase: every block in order
-                    if (fwd && a.indptr) {
-                        const int jr = a.kv_idx[it.begin + t];
-                        if (jr < 0 || jr >= a.nk) atomicOr(&g_device_error, kDevErrBadData);
+                    const bool fwd = t < it.tiles;
+                    const bool gather = fwd && SUB > 1 && a.indptr;  // C = 32 list: four 32-row blocks per tile
+                    int32_t krow = 0;
+                    if (!gather) {
+                        const int j = fwd ? (a.indptr ? list_block(a, it, t) : t) : t - it.tiles;
+                        krow = it.h * a.Np + j * kTcRows;
                     }
-                    const int32_t krow = it.h * a.Np + j * kTcRows;
+                    if (fwd && a.indptr) {
+                        for (int e = SUB * t; e < SUB * t + SUB && e < it.count; ++e) {
+                            const int jr = a.kv_idx[it.begin + e];
+                            if (jr < 0 || jr >= a.nkb) atomicOr(&g_device_error, kDevErrBadData);
+                        }
+                    }
                     if (!(ok = wait_bounded(BAR(L_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
                     mbar_arrive_expect_tx(BAR(L_K_FULL), kTileBytes);
-                    tma_load_2d_hint(sK, &tmK, 0, krow, BAR(L_K_FULL), pol_kv);
-                    tma_load_2d_hint(sK + kBoxBytes, &tmK, 64, krow, BAR(L_K_FULL), pol_kv);
+                    if (!gather) {
+                        tma_load_2d_hint(sK, &tmK, 0, krow, BAR(L_K_FULL), pol_kv);
+                        tma_load_2d_hint(sK + kBoxBytes, &tmK, 64, krow, BAR(L_K_FULL), pol_kv);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < SUB; ++g) {
+                            // a missing quarter reloads the tile's first block (finite data, masked to P = 0)
+                            const int e = SUB * t + g < it.count ? SUB * t + g : SUB * t;
+                            const int32_t r32 = it.h * a.Np + list_block(a, it, e) * 32;
+                            tma_load_2d_hint(sK + g * 4096u, &tmK32, 0, r32, BAR(L_K_FULL), pol_kv);
+                            tma_load_2d_hint(sK + kBoxBytes + g * 4096u, &tmK32, 64, r32, BAR(L_K_FULL), pol_kv);
+                        }
+                    }
                     ++nk_ld;
                     if (fwd) {
                         if (!(ok = wait_bounded(BAR(L_V_EMPTY), (nv_ld & 1u) ^ 1u, lim))) break;
                         mbar_arrive_expect_tx(BAR(L_V_FULL), kTileBytes);
-                        tma_load_2d_hint(sV, &tmV, 0, krow, BAR(L_V_FULL), pol_kv);
-                        tma_load_2d_hint(sV + kBoxBytes, &tmV, 64, krow, BAR(L_V_FULL), pol_kv);
+                        if (!gather) {
+                            tma_load_2d_hint(sV, &tmV, 0, krow, BAR(L_V_FULL), pol_kv);
+                            tma_load_2d_hint(sV + kBoxBytes, &tmV, 64, krow, BAR(L_V_FULL), pol_kv);
+                        } else {
+#pragma unroll
+                            for (int g = 0; g < SUB; ++g) {
+                                const int e = SUB * t + g < it.count ? SUB * t + g : SUB * t;
+                                const int32_t r32 = it.h * a.Np + list_block(a, it, e) * 32;
+                                tma_load_2d_hint(sV + g * 4096u, &tmV32, 0, r32, BAR(L_V_FULL), pol_kv);
+                                tma_load_2d_hint(sV + kBoxBytes + g * 4096u, &tmV32, 64, r32, BAR(L_V_FULL), pol_kv);
+                            }
+                        }
                         ++nv_ld;
                     }
                 }
@@ -276,14 +332,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (it.count <= 0) continue;
                 if (!(ok = wait_bounded(BAR(L_Q_FULL), nq & 1u, lim))) break;
                 ++nq;
-                const int total = it.count + mass_tiles;
+                const int total = it.tiles + mass_tiles;
                 for (int t = 0; t < total; ++t) {
-                    const bool fwd = t < it.count;
+                    const bool fwd = t < it.tiles;
                     if (!(ok = wait_bounded(BAR(L_K_FULL), nk_use & 1u, lim))) break;
                     // The S/P columns are free once the previous tile's P V (forward) or S read (mass) completed.
-                    if (t > 0 && t <= it.count) {
+                    if (t > 0 && t <= it.tiles) {
                         if (!(ok = wait_bounded(BAR(L_PV_DONE), (n_pv - 1) & 1u, lim))) break;
-                    } else if (t > it.count) {
+                    } else if (t > it.tiles) {
                         if (!(ok = wait_bounded(BAR(L_S_FREE), (n_sfree - 1) & 1u, lim))) break;
                     } else if (n_items > 0) {
                         // first tile of an item: the previous item's last S/P use must be over
@@ -333,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t lane_off = (wl * 32u) << 16;
         const float c = a.scale_log2;
         float* const part = reinterpret_cast<float*>(base_ptr + part_off + x * kPartBytes);
-        uint32_t n_s = 0, n_pv = 0, n_items = 0;
+        uint32_t n_s = 0, n_pv = 0, n_items = 0, n_chunks = 0;
         bool ok = true;
         ItemInfo it;
         for (int r = (int)x; ok && item_of_round(a, r, it); r += 2) {
@@ -341,14 +397,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int qrow = it.qb * kTcRows + row;
             const size_t grow = (size_t)it.h * a.Np + qrow;
             float m_raw = -INFINITY, l_run = 0.0f;
-            int jn = fwd_block(a, it, 0);
-            for (int t = 0; t < it.count; ++t) {
-                const int j = jn;
-                if (t + 1 < it.count) jn = fwd_block(a, it, t + 1);  // prefetch the next block index
+            uint32_t kvn = quarter_keys<SUB>(a, it, 0);
+            for (int t = 0; t < it.tiles; ++t) {
+                const uint32_t kv4 = kvn;  // real keys per 32-column quarter of this tile
+                if (t + 1 < it.tiles) kvn = quarter_keys<SUB>(a, it, t + 1);  // prefetched one tile ahead
+                const bool full = kv4 == 0x20202020u;
                 if (!(ok = wait_bounded_warp(BAR(L_S_FULL), n_s & 1u, lim))) break;
                 ++n_s;
                 tc_fence_after();
-                const int kvalid = a.N - j * kTcRows;  // < 128 only in the ragged last key block
                 // Pass 1: the tile's row max over all 128 columns (only columns 0..31 stay live afterwards).
                 float s0[32];
                 float tmax;
@@ -358,10 +414,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int ch = 0; ch < 4; ++ch)
                         tmem_ld32(tS + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
                     tmem_wait_ld();
-                    if (kvalid < kTcRows) {  // keys t >= N do not exist
+                    if (!full) {  // keys past the sequence end, or quarters without a listed block, do not exist
 #pragma unroll
                         for (int cc = 0; cc < 128; ++cc)
-                            if (cc >= kvalid) s[cc] = -INFINITY;
+                            if ((uint32_t)(cc & 31) >= ((kv4 >> (8 * (cc >> 5))) & 255u)) s[cc] = -INFINITY;
                     }
                     float mx[8];
 #pragma unroll
@@ -376,8 +432,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 // Reference max: raised only when the tile max exceeds it by more than 2^8 in the exp2 domain.
                 const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
-                const float alpha = (t > 0 && need) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
-                if (need) m_raw = tmax;
+                const float alpha = (t > 0 && need && tmax != -INFINITY) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
+                // A tile without any real key (only possible for a listed block that is all padding) keeps a finite
+                // reference so that its weights come out as exact zeros.
+                if (need) m_raw = (tmax == -INFINITY) ? (t == 0 ? 0.0f : m_raw) : tmax;
                 const float neg_mc = -m_raw * c;
                 // Pass 2, 32 columns at a time, the next chunk's TMEM load in flight during this chunk's math:
                 // P = 2^(s*c - m*c) as bf16 pairs written behind the read position (columns 16*ch .. 16*ch + 15
@@ -390,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tmem_ld32(tS + lane_off + (ch + 1) * 32u, *reinterpret_cast<uint32_t(*)[32]>(&rb[(ch + 1) & 1][0]));
                     const float* r = (ch == 0) ? s0 : rb[ch & 1];
                     uint32_t pw[16];
-                    if (kvalid >= kTcRows) {
+                    if (full) {
                         // three pairs in eight on the FMA pipe (packed polynomial), the rest on the exp unit
                         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
 #pragma unroll
@@ -410,10 +468,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                     } else {
 #pragma unroll
+                        const int kq = (int)((kv4 >> (8 * ch)) & 255u);  // chunk ch is quarter ch
                         for (int e = 0; e < 16; ++e) {
-                            const int c0 = ch * 32 + 2 * e;
-                            const float p0 = (c0 < kvalid) ? ex2_approx(fmaf(r[2 * e], c, neg_mc)) : 0.0f;
-                            const float p1 = (c0 + 1 < kvalid) ? ex2_approx(fmaf(r[2 * e + 1], c, neg_mc)) : 0.0f;
+                            const float p0 = (2 * e < kq) ? ex2_approx(fmaf(r[2 * e], c, neg_mc)) : 0.0f;
+                            const float p1 = (2 * e + 1 < kq) ? ex2_approx(fmaf(r[2 * e + 1], c, neg_mc)) : 0.0f;
                             pw[e] = pack_bf16x2(p0, p1);
                             l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                         }
@@ -444,8 +502,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (!ok) break;
             // Epilogue: O / l -> bf16 rows and lse; O's columns are then free for the next item.
-            if (!(ok = wait_bounded_warp(BAR(L_PV_DONE), (n_pv + it.count - 1) & 1u, lim))) break;
-            n_pv += it.count;
+            if (!(ok = wait_bounded_warp(BAR(L_PV_DONE), (n_pv + it.tiles - 1) & 1u, lim))) break;
+            n_pv += it.tiles;
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
             const float lse2 = m_raw * c + lg2_approx(l_run);
@@ -470,68 +528,97 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (a.lse) a.lse[grow] = lse2 * 0.6931471805599453f;
 
             if (WITH_MASS) {
-                // Mass phase: p = 2^(s*c - lse2) summed per key block for real rows and real keys.
+                // Mass phase: p = 2^(s*c - lse2) summed per key block (SUB blocks per tile) for real rows and keys.
+                // The per-warp partials are flushed to M every kMaxMassBlocks blocks: all 128 threads arrive on PART
+                // once their partials are written, combine the four warps in fixed order, then arrive on PART2 before
+                // the buffer is written again.
                 const bool qvalid = qrow < a.N;
                 const float neg_lse2 = qvalid ? -lse2 : 0.0f;
-                for (int j = 0; j < a.nk; ++j) {
-                    if (!(ok = wait_bounded_warp(BAR(L_S_FULL), n_s & 1u, lim))) break;
-                    ++n_s;
-                    tc_fence_after();
-                    float s[128];
+                const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(neg_lse2, neg_lse2);
+                const float inv_rows = 1.0f / (float)min(kTcRows, a.N - it.qb * kTcRows);
+                float* mrow = a.mass + (size_t)it.id * a.nkb;
+                constexpr int kChunkTiles = kMaxMassBlocks / SUB;
+                for (int t0 = 0; ok && t0 < a.nk; t0 += kChunkTiles) {
+                    const int t1 = min(a.nk, t0 + kChunkTiles);
+                    for (int t = t0; t < t1; ++t) {
+                        if (!(ok = wait_bounded_warp(BAR(L_S_FULL), n_s & 1u, lim))) break;
+                        ++n_s;
+                        tc_fence_after();
+                        float s[128];
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-                        tmem_ld32(tS + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(BAR(L_S_FREE));
-                    const int kvalid = a.N - j * kTcRows;
-                    uint64_t acc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-                    const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(neg_lse2, neg_lse2);
-                    if (kvalid >= kTcRows) {
-                        // seven pairs in sixteen on the FMA pipe (packed polynomial), the rest on the exp unit
+                        for (int ch = 0; ch < 4; ++ch)
+                            tmem_ld32(tS + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        mbar_arrive(BAR(L_S_FREE));
+                        const int kvalid = a.N - t * kTcRows;
+                        // acc[2 * g + (e & 1)]: two packed accumulators per 32-key quarter g
+                        uint64_t acc[8];
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) {
-                            const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nl2);
-                            float p0, p1;
-                            if ((e & 15) >= 9) {
-                                exp2_poly2(xx, p0, p1);
-                            } else {
-                                float x0, x1;
-                                f2_unpack(xx, x0, x1);
-                                p0 = ex2_approx(x0);
-                                p1 = ex2_approx(x1);
+                        for (int i = 0; i < 8; ++i) acc[i] = f2_pack(0.f, 0.f);
+                        if (kvalid >= kTcRows) {
+                            // seven pairs in sixteen on the FMA pipe (packed polynomial), the rest on the exp unit
+#pragma unroll
+                            for (int e = 0; e < 64; ++e) {
+                                const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nl2);
+                                float p0, p1;
+                                if ((e & 15) >= 9) {
+                                    exp2_poly2(xx, p0, p1);
+                                } else {
+                                    float x0, x1;
+                                    f2_unpack(xx, x0, x1);
+                                    p0 = ex2_approx(x0);
+                                    p1 = ex2_approx(x1);
+                                }
+                                acc[2 * (e >> 4) + (e & 1)] = f2_add(acc[2 * (e >> 4) + (e & 1)], f2_pack(p0, p1));
                             }
-                            acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
-                        }
-                    } else {
+                        } else {
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) {
-                            const float p0 = (2 * e < kvalid) ? ex2_approx(fmaf(s[2 * e], c, neg_lse2)) : 0.0f;
-                            const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_lse2)) : 0.0f;
-                            acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+                            for (int e = 0; e < 64; ++e) {
+                                const float p0 = (2 * e < kvalid) ? ex2_approx(fmaf(s[2 * e], c, neg_lse2)) : 0.0f;
+                                const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_lse2)) : 0.0f;
+                                acc[2 * (e >> 4) + (e & 1)] = f2_add(acc[2 * (e >> 4) + (e & 1)], f2_pack(p0, p1));
+                            }
+                        }
+                        float q[4];
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            float x0, x1, x2, x3;
+                            f2_unpack(acc[2 * g], x0, x1);
+                            f2_unpack(acc[2 * g + 1], x2, x3);
+                            q[g] = qvalid ? (x0 + x1) + (x2 + x3) : 0.0f;
+                        }
+                        if (SUB == 1) {
+                            float sum = (q[0] + q[1]) + (q[2] + q[3]);
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                            if (lane == 0) part[wl * kMaxMassBlocks + (t - t0)] = sum;
+                        } else {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+#pragma unroll
+                                for (int o = 16; o > 0; o >>= 1) q[g] += __shfl_xor_sync(0xffffffffu, q[g], o);
+                            }
+                            if (lane < 4) {
+                                const float mine = lane == 0 ? q[0] : (lane == 1 ? q[1] : (lane == 2 ? q[2] : q[3]));
+                                part[wl * kMaxMassBlocks + (t - t0) * SUB + lane] = mine;
+                            }
                         }
                     }
-                    float a0, a1, a2, a3, a4, a5, a6, a7;
-                    f2_unpack(acc[0], a0, a1);
-                    f2_unpack(acc[1], a2, a3);
-                    f2_unpack(acc[2], a4, a5);
-                    f2_unpack(acc[3], a6, a7);
-                    float sum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-                    if (!qvalid) sum = 0.0f;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                    if (lane == 0) part[wl * kMaxMassBlocks + j] = sum;
+                    if (!ok) break;
+                    mbar_arrive(BAR(L_PART));
+                    if (!(ok = wait_bounded_warp(BAR(L_PART), n_chunks & 1u, lim))) break;
+                    const int b0 = t0 * SUB, b1 = min(a.nkb, t1 * SUB);
+                    for (int jj = b0 + row; jj < b1; jj += 128) {
+                        const int o = jj - b0;
+                        mrow[jj] = ((part[o] + part[kMaxMassBlocks + o]) +
+                                    (part[2 * kMaxMassBlocks + o] + part[3 * kMaxMassBlocks + o])) * inv_rows;
+                    }
+                    mbar_arrive(BAR(L_PART2));
+                    if (!(ok = wait_bounded_warp(BAR(L_PART2), n_chunks & 1u, lim))) break;
+                    ++n_chunks;
                 }
                 if (!ok) break;
-                // The four warps' partial sums are complete once all 128 threads have arrived. The next item's
-                // partials are written only after every thread has passed its forward tiles, i.e. after this read.
-                mbar_arrive(BAR(L_PART));
-                if (!(ok = wait_bounded_warp(BAR(L_PART), n_items & 1u, lim))) break;
-                const float inv_rows = 1.0f / (float)min(kTcRows, a.N - it.qb * kTcRows);
-                float* mrow = a.mass + (size_t)it.id * a.nk;
-                for (int jj = row; jj < a.nk; jj += 128)
-                    mrow[jj] = ((part[jj] + part[kMaxMassBlocks + jj]) +
-                                (part[2 * kMaxMassBlocks + jj] + part[3 * kMaxMassBlocks + jj])) * inv_rows;
             }
             ++n_items;
         }

@@ -42,16 +42,20 @@ losa_status check_shape(const losa_shape* s) {
         return LOSA_ERR_INVALID_ARG;
     if (s->n_padded < s->n_tokens || s->n_padded % s->block_q != 0 || s->n_padded % s->block_k != 0)
         return LOSA_ERR_INVALID_ARG;
-    // Every block must hold at least one real token.
-    if (s->n_padded - s->n_tokens >= s->block_q || s->n_padded - s->n_tokens >= s->block_k)
-        return LOSA_ERR_INVALID_ARG;
+    // Every query block must hold at least one real row. Key blocks smaller than the query blocks may lie entirely in
+    // the padding (they then carry zero mass and are never selected).
+    if (s->n_padded - s->n_tokens >= s->block_q) return LOSA_ERR_INVALID_ARG;
+    if (s->block_k >= s->block_q && s->n_padded - s->n_tokens >= s->block_k) return LOSA_ERR_INVALID_ARG;
     if (s->dtype != LOSA_DTYPE_BF16 && s->dtype != LOSA_DTYPE_F32) return LOSA_ERR_INVALID_ARG;
     if ((long long)s->heads * s->n_padded * s->head_dim > (1ll << 40)) return LOSA_ERR_INVALID_ARG;
     return LOSA_OK;
 }
 
+// Tensor-core path: bf16, head_dim 128, query blocks of 128 rows, key blocks of 128 or 32 keys (the LoSA page's
+// experimental setup uses R = 128, C = 32), at most 1024 tiles of 128 keys per head.
 bool tc_shape(const losa_shape* s) {
-    return s->dtype == LOSA_DTYPE_BF16 && s->head_dim == kTcDim && s->block_q == kTcRows && s->block_k == kTcRows &&
+    return s->dtype == LOSA_DTYPE_BF16 && s->head_dim == kTcDim && s->block_q == kTcRows &&
+           (s->block_k == kTcRows || s->block_k == 32) && s->n_padded % kTcRows == 0 &&
            s->n_padded / kTcRows <= kMaxMassBlocks;
 }
 
@@ -90,17 +94,28 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Tensor map over a [rows][128] bf16 matrix, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows) {
+// Tensor map over a [rows][128] bf16 matrix, boxes of box_rows rows x 64 columns, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t box_rows = kTcRows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t gdim[2] = {(cuuint64_t)kTcDim, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)kTcDim * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kTcRows};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estride[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box, estride,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool M, int SUB>
+losa_status launch_tc_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tk32, const CUtensorMap& tv32, const TcArgs& a, cudaStream_t stream) {
+    const uint32_t smem = tc_smem_bytes<M>();
+    if (cudaFuncSetAttribute(attn_tc_kernel<M, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    attn_tc_kernel<M, SUB><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, tk32, tv32, a);
+    return launch_status();
 }
 
 // Tensor-core path: fills the argument block and launches one persistent CTA (two lanes) per SM.
@@ -108,15 +123,22 @@ losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const 
                       const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
                       float* mass, cudaStream_t stream) {
     const uint64_t rows = (uint64_t)s->heads * s->n_padded;
-    CUtensorMap tq, tk, tv;
+    const bool c32 = s->block_k == 32;
+    CUtensorMap tq, tk, tv, tk32, tv32;
     if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
         return LOSA_ERR_CUDA;
+    if (c32 && (!make_tile_map(&tk32, k, rows, 32) || !make_tile_map(&tv32, v, rows, 32))) return LOSA_ERR_CUDA;
+    if (!c32) {
+        tk32 = tk;
+        tv32 = tv;
+    }
     TcArgs a;
     a.H = s->heads;
     a.N = s->n_tokens;
     a.Np = s->n_padded;
     a.nq = s->n_padded / kTcRows;
     a.nk = s->n_padded / kTcRows;
+    a.nkb = s->n_padded / s->block_k;
     a.n_items = s->heads * a.nq;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.indptr = indptr;
@@ -130,20 +152,11 @@ losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const 
     if (sms <= 0) return LOSA_ERR_CUDA;
     const int want = (a.n_items + 1) / 2;  // two lanes per CTA
     const int grid = want < sms ? (want > 0 ? want : 1) : sms;
-    if (with_mass) {
-        const uint32_t smem = tc_smem_bytes<true>();
-        if (cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return LOSA_ERR_CUDA;
-        attn_tc_kernel<true><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
-    } else {
-        const uint32_t smem = tc_smem_bytes<false>();
-        if (cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return LOSA_ERR_CUDA;
-        attn_tc_kernel<false><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, a);
-    }
-    return launch_status();
+    if (with_mass)
+        return c32 ? launch_tc_kernel<true, 4>(grid, tq, tk, tv, tk32, tv32, a, stream)
+                   : launch_tc_kernel<true, 1>(grid, tq, tk, tv, tk32, tv32, a, stream);
+    return c32 ? launch_tc_kernel<false, 4>(grid, tq, tk, tv, tk32, tv32, a, stream)
+               : launch_tc_kernel<false, 1>(grid, tq, tk, tv, tk32, tv32, a, stream);
 }
 
 template <int D>

@@ -34,12 +34,13 @@ class LayerBuffers:
     block: int
     dtype: str
     device: str = "cuda"
+    block_k: int = 0  # key block size when it differs from the query block size
 
     def __post_init__(self):
-        self.shape = make_shape(self.heads, self.n_tokens, self.n_padded, self.head_dim, self.block, self.block,
-                                self.dtype)
+        bk = self.block_k or self.block
+        self.shape = make_shape(self.heads, self.n_tokens, self.n_padded, self.head_dim, self.block, bk, self.dtype)
         self.nq = self.n_padded // self.block
-        self.nk = self.nq
+        self.nk = self.n_padded // bk
         self.rows = self.heads * self.nq
         tdt = torch.bfloat16 if self.dtype == "bf16" else torch.float32
         dev = self.device
@@ -54,7 +55,8 @@ class LayerBuffers:
 
     @classmethod
     def for_config(cls, cfg, device="cuda"):
-        return cls(cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block, cfg.dtype, device)
+        return cls(cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block, cfg.dtype, device,
+                   getattr(cfg, "block_k", 0))
 
     def profile(self, q, k, v, scale, with_mass=True, stream=None):
         losa_dense_profile(self.shape, q, k, v, scale, self.o, self.lse, self.mass if with_mass else None,

@@ -14,7 +14,7 @@
  *     synchronises the stream). Host-side argument checks run first and return before anything is launched.
  *   - Token tensors q, k, v, o are [H][Np][d] row-major, d contiguous: head h, token t starts at element
  *     (h * Np + t) * d. Tokens are the video latent's (t, y, x) grid flattened row-major, padded from N to Np
- *     (a multiple of the block sizes, N <= Np < N + block). Keys t >= N take no part in any softmax; output
+ *     (a multiple of the block sizes, N <= Np < N + block_q). Keys t >= N take no part in any softmax; output
  *     rows t >= N are written but carry no meaning. Base pointers must be 16-byte aligned.
  *   - An "item" is one (head, query block) pair with id h * nq + i, nq = Np / block_q, nk = Np / block_k.
  *   - A batch (several samples, or the conditional and unconditional branches of classifier-free guidance) is passed
@@ -22,8 +22,9 @@
  *     page's Methodology Summary keeps separate patterns for the two guidance branches.
  *   - Status codes below; LOSA_ERR_CUDA covers launch failures reported by the CUDA runtime.
  *
- * Supported shapes: dtype BF16 with head_dim 128 and block_q = block_k = 128 (tensor-core path), or dtype F32
- * with head_dim 64 or 128 and block_q = block_k in {32, 64, 128} (exact fp32 path for small checks).
+ * Supported shapes: dtype BF16 with head_dim 128, block_q = 128 and block_k = 128 or 32 (tensor-core path; 32 is the
+ * LoSA page's key-block size), or dtype F32 with head_dim 64 or 128 and block_q = block_k in {32, 64, 128} (exact fp32
+ * path for small checks).
  */
 #ifndef LOSA_H
 #define LOSA_H
@@ -51,7 +52,7 @@ enum { LOSA_DTYPE_F32 = 0, LOSA_DTYPE_BF16 = 1 };
 typedef struct {
     int32_t heads;     /* H                                                        */
     int32_t n_tokens;  /* N, real tokens                                            */
-    int32_t n_padded;  /* Np, multiple of block_q and block_k, N <= Np < N + block  */
+    int32_t n_padded;  /* Np, multiple of block_q and block_k, N <= Np < N + block_q */
     int32_t head_dim;  /* d                                                        */
     int32_t block_q;   /* R, query block size                                       */
     int32_t block_k;   /* C, key/value block size                                   */

@@ -40,7 +40,7 @@ class LayerConfig:
     heads: int
     grid: tuple            # (T, Y, X) token grid; N = T*Y*X, flattened row-major (t, y, x)
     head_dim: int
-    block: int             # query block size R = key/value block size C
+    block: int             # query block size R (and key/value block size C unless block_k is set)
     dtype: str             # "f32" or "bf16"
     amplitude: float       # a
     ell_fixed: tuple | None = None      # per-axis lengthscale (t, y, x), or None
@@ -52,6 +52,15 @@ class LayerConfig:
     layers: int = 1
     taus: tuple = (0.99,)
     extra: dict = field(default_factory=dict)
+    block_k: int = 0       # key/value block size C when it differs from R (the LoSA page's setup: R = 128, C = 32)
+
+    @property
+    def kblock(self) -> int:
+        return self.block_k or self.block
+
+    @property
+    def n_kblocks(self) -> int:
+        return self.n_padded // self.kblock
 
     @property
     def n_tokens(self) -> int:

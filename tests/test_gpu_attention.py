@@ -37,6 +37,14 @@ SMALL = {
                                              dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=1,
                                              seed=102, taus=(0.99,)),
     "f32-tiny": CONFIGS[0],
+    # the LoSA page's block shape: 128-row query blocks, 32-key blocks
+    "bf16-C32-2x(4x16x16)": LayerConfig("small-bf16-c32", heads=2, grid=(4, 16, 16), head_dim=128, block=128,
+                                        block_k=32, dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=2,
+                                        seed=103, taus=(0.5, 0.9, 0.99, 1.0)),
+    # 2015 tokens padded to 2048: the last 32-key block is all padding
+    "bf16-C32-3x(5x13x31)-ragged": LayerConfig("ragged-bf16-c32", heads=3, grid=(5, 13, 31), head_dim=128,
+                                               block=128, block_k=32, dtype="bf16", amplitude=4.0,
+                                               ell_range=(1.0, 8.0), n_sinks=2, seed=104, taus=(0.9, 0.99, 1.0)),
 }
 
 
@@ -50,7 +58,7 @@ def _pipeline(cfg, items, oracle, layer=None):
     qf, kf, vf = layer.all_f32("q"), layer.all_f32("k"), layer.all_f32("v")
     if items is None:
         items = np.arange(buf.rows, dtype=np.int32)
-    R, N = cfg.block, cfg.n_tokens
+    R, C, N = cfg.block, cfg.kblock, cfg.n_tokens
 
     # dense forward
     od, ld = oracle.dense(qf, kf, vf, N, R, scale, items)
@@ -61,7 +69,7 @@ def _pipeline(cfg, items, oracle, layer=None):
 
     # block masses
     gm_all = buf.mass.cpu().numpy().reshape(buf.rows, buf.nk)
-    om = oracle.mass(qf, kf, N, R, R, scale, items)
+    om = oracle.mass(qf, kf, N, R, C, scale, items)
     check_mass(gm_all[items], om, f"{cfg.name}")
     np.testing.assert_allclose(gm_all.sum(axis=1), 1.0, atol=1e-3)
 
@@ -79,7 +87,7 @@ def _pipeline(cfg, items, oracle, layer=None):
         l2 = torch.empty_like(buf.lse)
         buf.sparse(q, k, v, scale, out=o2, lse=l2)
         assert L.losa_get_device_error() == 0
-        os_, ls_ = oracle.sparse(qf, kf, vf, N, R, R, scale, gi, gk, items)
+        os_, ls_ = oracle.sparse(qf, kf, vf, N, R, C, scale, gi, gk, items)
         go2, _ = item_rows(cfg, items, o2.float().cpu().numpy())
         gl2, _ = item_rows(cfg, items, l2.cpu().numpy())
         check_output(go2[valid], os_[valid], f"{cfg.name} sparse O tau={tau}")
@@ -92,9 +100,10 @@ def test_small_full_comparison(name, oracle_mod):
     _pipeline(SMALL[name], None, oracle_mod)
 
 
-@pytest.mark.parametrize("cfg_id", [1, 2, 3])
-def test_full_size_sampled(cfg_id, oracle_mod):
-    cfg = CONFIGS[cfg_id]
+@pytest.mark.parametrize("cfg_id,block_k", [(1, 128), (2, 128), (3, 128), (1, 32), (3, 32)])
+def test_full_size_sampled(cfg_id, block_k, oracle_mod):
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS[cfg_id], block_k=block_k)
     layer = make_layer(cfg)
     # 64 seeded items, including the tail block of head 0 and the query blocks holding head 0's sink tokens
     sink_items = [int(t) // cfg.block for t in layer.sinks[0]]
