@@ -21,6 +21,7 @@ constexpr unsigned int kDevErrBadData = 2u;
 
 #include "attn_f32.cuh"
 #include "attn_tc.cuh"
+#include "attn_dense.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
 
@@ -108,6 +109,16 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t bo
 }
 
 template <bool M, int SUB>
+losa_status launch_dense_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const TcArgs& a, cudaStream_t stream) {
+    if (cudaFuncSetAttribute(attn_dense_kernel<M, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDnSmem) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    attn_dense_kernel<M, SUB><<<grid, kTcThreads, kDnSmem, stream>>>(tq, tk, tv, a);
+    return launch_status();
+}
+
+template <bool M, int SUB>
 losa_status launch_tc_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tk32, const CUtensorMap& tv32, const TcArgs& a, cudaStream_t stream) {
     const uint32_t smem = tc_smem_bytes<M>();
@@ -150,6 +161,15 @@ losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const 
     a.wait_limit_ns = g_wait_limit_ns;
     const int sms = sm_count();
     if (sms <= 0) return LOSA_ERR_CUDA;
+    if (!indptr) {
+        // dense step: one item per CTA at a time, 256-key tiles
+        const int dgrid = a.n_items < sms ? a.n_items : sms;
+        if (with_mass)
+            return c32 ? launch_dense_kernel<true, 4>(dgrid, tq, tk, tv, a, stream)
+                       : launch_dense_kernel<true, 1>(dgrid, tq, tk, tv, a, stream);
+        return c32 ? launch_dense_kernel<false, 4>(dgrid, tq, tk, tv, a, stream)
+                   : launch_dense_kernel<false, 1>(dgrid, tq, tk, tv, a, stream);
+    }
     const int want = (a.n_items + 1) / 2;  // two lanes per CTA
     const int grid = want < sms ? (want > 0 ? want : 1) : sms;
     if (with_mass)

@@ -124,10 +124,12 @@ def test_sparse_with_every_block_equals_dense():
     o2 = torch.empty_like(buf.o)
     buf.sparse(q, k, v, scale, out=o2, order=False)
     assert L.losa_get_device_error() == 0
+    # Two different kernels (256-key tiles vs 128-key tiles, different running-max references) each round O to bf16;
+    # they must agree within the output tolerance both meet against the fp64 oracle.
     n = cfg.n_tokens
-    a = buf.o[:, :n].float()
-    b = o2[:, :n].float()
-    assert (a - b).abs().max().item() <= 1e-2
+    a = buf.o[:, :n].float().cpu().numpy().reshape(-1, cfg.head_dim)
+    b = o2[:, :n].float().cpu().numpy().reshape(-1, cfg.head_dim)
+    check_output(b, a.astype(np.float64), "full-list sparse vs dense")
 
 
 def test_sparse_random_lists_and_orders(oracle_mod):
