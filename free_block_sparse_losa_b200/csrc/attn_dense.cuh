@@ -42,13 +42,13 @@ template <bool WITH_MASS, int SUB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_dense_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t base = smem_addr(smem_raw);
+    extern __shared__ __align__(1024) uint8_t dn_smem[];
+    const uint32_t base = smem_addr(dn_smem);
     if (base & 1023u) {  // the 128-byte-swizzled tiles need a 1024-aligned base; report instead of overrunning
         if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrBadData);
         return;
     }
-    uint8_t* const base_ptr = smem_raw;
+    uint8_t* const base_ptr = dn_smem;
     const uint32_t bar0 = base + kDnBar;
     auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kDnBar + D_COUNT * 8);
@@ -214,19 +214,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!(ok = wait_bounded_warp(BAR(D_S_FULL), n_s & 1u, lim))) break;
                 ++n_s;
                 tc_fence_after();
-                // Pass 1: this group's row max, exchanged with the other group.
+                // One TMEM read of this group's 128 columns. S is released at once, so the next QK^T runs under
+                // this tile's softmax.
+                float s[128];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)
+                    tmem_ld32(tSg + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(BAR(D_S_FREE));
+                if (!full) {
+#pragma unroll
+                    for (int cc = 0; cc < 128; ++cc)
+                        if (cc >= kvalid) s[cc] = -INFINITY;
+                }
                 float tmax;
                 {
-                    float s[128];
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-                        tmem_ld32(tSg + lane_off + ch * 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[ch * 32]));
-                    tmem_wait_ld();
-                    if (!full) {
-#pragma unroll
-                        for (int cc = 0; cc < 128; ++cc)
-                            if (cc >= kvalid) s[cc] = -INFINITY;
-                    }
                     float mx[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) mx[e] = fmax3(s[e], s[8 + e], s[16 + e]);
@@ -236,59 +239,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], s[cc + e], s[cc + 8 + e]);
                     tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
                 }
+                // The row max over both groups' columns, exchanged through shared memory.
                 float* xm = xmax + (n_x & 1u) * 256u;
                 xm[grp * 128u + row] = tmax;
                 mbar_arrive(BAR(D_MAX_X));
                 if (!(ok = wait_bounded_warp(BAR(D_MAX_X), n_x & 1u, lim))) break;
                 ++n_x;
-                tmax = fmaxf(tmax, xm[(1u - grp) * 128u + row]);  // the tile max over all 256 columns
+                tmax = fmaxf(tmax, xm[(1u - grp) * 128u + row]);
                 const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
                 const float alpha = (t > 0 && need) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
                 if (need) m_raw = tmax;
                 const float neg_mc = -m_raw * c;
-                // Pass 2: P for this group's 128 columns, held in registers until the P unit is free.
+                // P for this group's 128 columns, from registers, held until the P unit is free.
                 uint32_t pw[64];
                 uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-                float rb[2][32];
-                tmem_ld32(tSg + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&rb[0][0]));
-                tmem_wait_ld_regs(rb[0]);
+                if (full) {
+                    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    if (ch < 3)
-                        tmem_ld32(tSg + lane_off + (ch + 1) * 32u, *reinterpret_cast<uint32_t(*)[32]>(&rb[(ch + 1) & 1][0]));
-                    const float* r = rb[ch & 1];
-                    if (full) {
-                        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const uint64_t xx = f2_fma(f2_pack(r[2 * e], r[2 * e + 1]), c2, nm2);
-                            float p0, p1;
-                            if ((e & 7) >= 5) {
-                                exp2_poly2(xx, p0, p1);
-                            } else {
-                                float x0, x1;
-                                f2_unpack(xx, x0, x1);
-                                p0 = ex2_approx(x0);
-                                p1 = ex2_approx(x1);
-                            }
-                            pw[ch * 16 + e] = pack_bf16x2(p0, p1);
-                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                    for (int e = 0; e < 64; ++e) {
+                        const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
+                        float p0, p1;
+                        if ((e & 7) >= 5) {
+                            exp2_poly2(xx, p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(xx, x0, x1);
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
                         }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int c0 = ch * 32 + 2 * e;
-                            const float p0 = (c0 < kvalid) ? ex2_approx(fmaf(r[2 * e], c, neg_mc)) : 0.0f;
-                            const float p1 = (c0 + 1 < kvalid) ? ex2_approx(fmaf(r[2 * e + 1], c, neg_mc)) : 0.0f;
-                            pw[ch * 16 + e] = pack_bf16x2(p0, p1);
-                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
-                        }
+                        pw[e] = pack_bf16x2(p0, p1);
+                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                     }
-                    if (ch < 3) tmem_wait_ld_regs(rb[(ch + 1) & 1]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) {
+                        const float p0 = (2 * e < kvalid) ? ex2_approx(fmaf(s[2 * e], c, neg_mc)) : 0.0f;
+                        const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_mc)) : 0.0f;
+                        pw[e] = pack_bf16x2(p0, p1);
+                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                    }
                 }
-                // S has been read: the next QK^T may overwrite it.
-                tc_fence_before();
-                mbar_arrive(BAR(D_S_FREE));
                 float la, lb, lc, ld;
                 f2_unpack(l2[0], la, lb);
                 f2_unpack(l2[1], lc, ld);

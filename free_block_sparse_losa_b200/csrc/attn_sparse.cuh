@@ -1,0 +1,533 @@
+// Sparse-step tensor-core kernel (bf16, head_dim 128, 128-row query blocks): attn_sparse_kernel<SUB>.
+//
+// Online-softmax attention of each work item = (head, 128-row query block) against its retained list of key blocks
+// (LoSA page, Methodology Summary, "Sparse attention with a frozen pattern": the softmax denominator covers the
+// retained keys only), SUB key blocks per 128-key tile (1 for C = 128, 4 for C = 32). Writes O (bf16) and the row
+// log-sum-exp.
+//
+// One persistent CTA per SM walks one stream of items (CTA b takes rounds r = 0, 1, 2, ...: item r*G + b for even r,
+// r*G + G - 1 - b for odd r, a snake over the longest-first work order). The tiles of all its items form one
+// sequence n = 0, 1, 2, ... through a software pipeline:
+//   warp 3   reads the work order and the lists ahead of time into a four-entry ring of item records in shared
+//            memory (head, query block, list start and length, tiles, key validity of the first tile), so that no
+//            role waits on dependent global loads at an item boundary.
+//   warp 0   TMA: Q double-buffered (the next item's Q arrives during this item), K in a three-stage ring.
+//   warp 2   TMA: V in a two-stage ring (a V slot waiting for its P V never holds back K).
+//   warp 1   MMA: at an item's start, Q is copied from shared memory into TMEM (tcgen05.cp); then per tile
+//            S_n = Q K^T (128 x 128, N = 128, Q read from TMEM) and O += P V of tile n - 1 (P from TMEM). With both
+//            A operands in TMEM, the MMAs read only K and V from shared memory.
+//   warps 4..11  softmax in two warpgroups that split each tile's keys (warps 4..7 keys 0..63, warps 8..11 keys
+//            64..127; thread t owns query row t = TMEM lane t). A group reads its half of S once and releases it, so
+//            the next QK^T runs under this tile's exponentials; the groups exchange their half-tile row maxima
+//            through shared memory, share one running max, keep their own partial sums and write their half of P.
+// TMEM: S columns 0..127, O 128..255, P_0 256..319, P_1 320..383 (bf16 pairs), Q_0 384..447, Q_1 448..511 (bf16
+// pairs, one buffer per item parity). O is rescaled in place only when a row's running max grows by more than 2^8
+// (the final division by the sum taken against the same reference keeps this exact); each group rescales its own 64
+// columns of O.
+// Epilogue: O / l in bf16 is written, 128-byte swizzled, into the V slot the item's last P V has just released and
+// leaves through two TMA stores (one 64-column box per group); the V producer gets the slot back once the stores
+// have read it. Row stores from registers would put 32 rows into every warp-wide store.
+// Every wait is bounded in time (LOSA_ERR_TIMEOUT in the device error word, then a clean exit).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "attn_tc.cuh"
+
+namespace losa {
+
+constexpr uint32_t kSpQ = 0;                              // 2 Q tiles
+constexpr uint32_t kSpK = 2 * kTileBytes;                 // 3 K tiles
+constexpr uint32_t kSpV = 5 * kTileBytes;                 // 2 V tiles (the second use: O staging)
+constexpr uint32_t kSpBar = 7 * kTileBytes;               // 48 barrier slots; the last holds the TMEM address
+constexpr uint32_t kSpX = kSpBar + 384;                   // [2 tile parity][2 groups][128] fp32 row maxima (sums alias)
+constexpr uint32_t kSpRing = kSpX + 2 * 2 * 128 * 4;      // 4 item records of 32 bytes
+constexpr uint32_t kSpSmem = kSpRing + 4 * 32;            // 231936 bytes: needs a 1024-aligned dynamic base
+constexpr int kSpKStages = 3;
+constexpr uint32_t kSpRingSlots = 4;
+
+enum : uint32_t {
+    S_Q_FULL0 = 0, S_Q_EMPTY0 = 2, S_K_FULL0 = 4, S_K_EMPTY0 = 7, S_V_FULL0 = 10, S_V_EMPTY0 = 12, S_S_FULL = 14,
+    S_S_FREE = 16, S_P_FULL0 = 18, S_PV_DONE0 = 20, S_MAX_X = 22, S_SUM_X, S_O_FREE, S_ST_READY0, S_ST_READY1 = 26,
+    S_ST_DONE, S_IT_FULL0, S_IT_EMPTY0 = S_IT_FULL0 + kSpRingSlots, S_MMA_DONE = S_IT_EMPTY0 + kSpRingSlots, S_COUNT
+};
+constexpr int kSpThreads = 384;  // 12 warps: 0 Q/K TMA, 1 MMA, 2 V TMA, 3 work order, 4..11 softmax
+static_assert(S_COUNT <= 47, "barrier slots");
+
+struct SpItem {
+    int id, h, qb, begin, count, tiles;
+    uint32_t kv4;  // real keys per 32-key quarter of the first tile
+    int end;       // 1: past the end of this CTA's work
+};
+static_assert(sizeof(SpItem) == 32, "item record");
+
+// List entry e of an item as a block index (clamped; out-of-range entries are reported by the work-order reader).
+__device__ __forceinline__ int sp_block(const TcArgs& a, const SpItem& it, int e) {
+    const int j = a.kv_idx[it.begin + e];
+    return (j < 0) ? 0 : (j >= a.nkb ? a.nkb - 1 : j);
+}
+
+template <int SUB>
+__device__ __forceinline__ void sp_load_tile(const TcArgs& a, const SpItem& it, int t, uint32_t dst,
+                                             const CUtensorMap* tm, const CUtensorMap* tm32, uint32_t bar,
+                                             uint64_t pol) {
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    if (SUB == 1) {
+        const int32_t krow = it.h * a.Np + sp_block(a, it, t) * kTcRows;
+        tma_load_2d_hint(dst, tm, 0, krow, bar, pol);
+        tma_load_2d_hint(dst + kBoxBytes, tm, 64, krow, bar, pol);
+    } else {
+#pragma unroll
+        for (int g = 0; g < SUB; ++g) {
+            // a missing quarter reloads the tile's first block (finite data, masked to P = 0)
+            const int e = SUB * t + g < it.count ? SUB * t + g : SUB * t;
+            const int32_t r32 = it.h * a.Np + sp_block(a, it, e) * 32;
+            tma_load_2d_hint(dst + g * 4096u, tm32, 0, r32, bar, pol);
+            tma_load_2d_hint(dst + kBoxBytes + g * 4096u, tm32, 64, r32, bar, pol);
+        }
+    }
+}
+
+// Real keys in each 32-key quarter of tile t of a list item, packed 8 bits per quarter. A quarter with no list entry
+// (the tail of a C = 32 list) has none; the ragged end of the sequence cuts the last block.
+template <int SUB>
+__device__ __forceinline__ uint32_t sp_quarter_keys(const TcArgs& a, const SpItem& it, int t) {
+    uint32_t kv = 0;
+    if (SUB == 1) {
+        const int kvalid = a.N - sp_block(a, it, t) * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) kv |= (uint32_t)min(32, max(0, kvalid - 32 * g)) << (8 * g);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int e = SUB * t + g;
+            if (e < it.count) kv |= (uint32_t)min(32, max(0, a.N - sp_block(a, it, e) * 32)) << (8 * g);
+        }
+    }
+    return kv;
+}
+
+template <int SUB>
+__global__ void __launch_bounds__(kSpThreads, 1)
+    attn_sparse_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK32,
+                       const __grid_constant__ CUtensorMap tmV32, const __grid_constant__ CUtensorMap tmO,
+                       const TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t sp_smem[];
+    const uint32_t base = smem_addr(sp_smem);
+    if (base & 1023u) {  // the 128-byte-swizzled tiles need a 1024-aligned base; report instead of overrunning
+        if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrBadData);
+        return;
+    }
+    const uint32_t bar0 = base + kSpBar;
+    auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sp_smem + kSpBar + 47 * 8);
+    float* const xmax = reinterpret_cast<float*>(sp_smem + kSpX);  // [2 tile parity][2 groups][128]
+    SpItem* const ring = reinterpret_cast<SpItem*>(sp_smem + kSpRing);
+
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (uint32_t s = 0; s < S_COUNT; ++s) {
+            uint32_t cnt = 1;
+            if (s == S_S_FREE || s == S_P_FULL0 || s == S_P_FULL0 + 1 || s == S_MAX_X ||
+                s == S_SUM_X || s == S_O_FREE)
+                cnt = 256;
+            else if (s == S_ST_READY0 || s == S_ST_READY1)
+                cnt = 128;
+            else if (s >= S_IT_EMPTY0 && s < S_IT_EMPTY0 + kSpRingSlots)
+                cnt = 3 + 256;  // Q/K producer, V producer, MMA issuer, 256 softmax threads
+            mbar_init(BAR(s), cnt);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
+        if (SUB > 1) {
+            tma_prefetch_desc(&tmK32);
+            tma_prefetch_desc(&tmV32);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+    const uint32_t tS = tmem, tO = tmem + 128u, tP = tmem + 256u, tQ = tmem + 384u;
+    const unsigned long long lim = a.wait_limit_ns;
+
+    // Item record of round r from the ring (false on a timeout); every consumer thread arrives on its slot.
+    auto next_item = [&](int r, SpItem& it, bool warp_wide) -> bool {
+        const uint32_t sl = (uint32_t)r & (kSpRingSlots - 1);
+        const uint32_t par = ((uint32_t)r / kSpRingSlots) & 1u;
+        const bool ok = warp_wide ? wait_bounded_warp(BAR(S_IT_FULL0 + sl), par, lim)
+                                  : wait_bounded(BAR(S_IT_FULL0 + sl), par, lim);
+        if (!ok) return false;
+        const volatile SpItem* src = &ring[sl];
+        it.id = src->id;
+        it.h = src->h;
+        it.qb = src->qb;
+        it.begin = src->begin;
+        it.count = src->count;
+        it.tiles = src->tiles;
+        it.kv4 = src->kv4;
+        it.end = src->end;
+        mbar_arrive(BAR(S_IT_EMPTY0 + sl));
+        return true;
+    };
+
+    if (warp == 3) {
+        // ------------------------------------------------------------------------- work-order reader (lane 0)
+        if (lane == 0) {
+            uint32_t bad = 0;
+            for (int r = 0;; ++r) {
+                const uint32_t sl = (uint32_t)r & (kSpRingSlots - 1);
+                if (!wait_bounded(BAR(S_IT_EMPTY0 + sl), (((uint32_t)r / kSpRingSlots) & 1u) ^ 1u, lim)) break;
+                ItemInfo ii;
+                const bool has = item_of_round(a, r, ii);
+                SpItem it;
+                it.end = has ? 0 : 1;
+                it.id = has ? ii.id : 0;
+                it.h = has ? ii.h : 0;
+                it.qb = has ? ii.qb : 0;
+                it.begin = has ? ii.begin : 0;
+                it.count = has ? ii.count : 0;
+                it.tiles = has ? ii.tiles : 0;
+                it.kv4 = 0;
+                if (has) {
+                    if (it.count <= 0) bad = 1;
+                    for (int e = 0; e < it.count; ++e) {
+                        const int j = a.kv_idx[it.begin + e];
+                        bad |= (j < 0 || j >= a.nkb) ? 1u : 0u;
+                    }
+                    if (it.count > 0) it.kv4 = sp_quarter_keys<SUB>(a, it, 0);
+                }
+                volatile SpItem* dst = &ring[sl];
+                dst->id = it.id;
+                dst->h = it.h;
+                dst->qb = it.qb;
+                dst->begin = it.begin;
+                dst->count = it.count;
+                dst->tiles = it.tiles;
+                dst->kv4 = it.kv4;
+                dst->end = it.end;
+                mbar_arrive(BAR(S_IT_FULL0 + sl));
+                if (!has) break;
+            }
+            if (bad) atomicOr(&g_device_error, kDevErrBadData);
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        // ----------------------------------------------------------------------------- TMA producer: Q and K
+        if (lane == 0) {
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            uint32_t nq = 0, nk = 0;
+            bool ok = true;
+            SpItem it;
+            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
+                if (it.count <= 0) continue;
+                const uint32_t qs = nq & 1u;
+                if (!(ok = wait_bounded(BAR(S_Q_EMPTY0 + qs), ((nq >> 1) & 1u) ^ 1u, lim))) break;
+                const int32_t qrow = it.h * a.Np + it.qb * kTcRows;
+                mbar_arrive_expect_tx(BAR(S_Q_FULL0 + qs), kTileBytes);
+                tma_load_2d_hint(base + kSpQ + qs * kTileBytes, &tmQ, 0, qrow, BAR(S_Q_FULL0 + qs), pol_q);
+                tma_load_2d_hint(base + kSpQ + qs * kTileBytes + kBoxBytes, &tmQ, 64, qrow, BAR(S_Q_FULL0 + qs),
+                                 pol_q);
+                ++nq;
+                for (int t = 0; t < it.tiles; ++t) {
+                    const uint32_t ks = nk % kSpKStages;
+                    if (!(ok = wait_bounded(BAR(S_K_EMPTY0 + ks), ((nk / kSpKStages) & 1u) ^ 1u, lim))) break;
+                    sp_load_tile<SUB>(a, it, t, base + kSpK + ks * kTileBytes, &tmK, &tmK32, BAR(S_K_FULL0 + ks),
+                                      pol_kv);
+                    ++nk;
+                }
+            }
+            for (uint32_t i = 1; i <= 2 && i <= nq; ++i) {
+                const uint32_t n = nq - i;
+                wait_bounded(BAR(S_Q_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
+            }
+            for (uint32_t i = 1; i <= kSpKStages && i <= nk; ++i) {
+                const uint32_t n = nk - i;
+                wait_bounded(BAR(S_K_FULL0 + n % kSpKStages), (n / kSpKStages) & 1u, kDrainLimitNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ----------------------------------------------------------------------------------- TMA producer: V
+        if (lane == 0) {
+            const uint64_t pol_kv = l2_policy_evict_last();
+            uint32_t nv = 0;
+            bool ok = true;
+            SpItem it;
+            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
+                if (it.count <= 0) continue;
+                for (int t = 0; t < it.tiles; ++t) {
+                    const uint32_t vs = nv & 1u;
+                    if (!(ok = wait_bounded(BAR(S_V_EMPTY0 + vs), ((nv >> 1) & 1u) ^ 1u, lim))) break;
+                    sp_load_tile<SUB>(a, it, t, base + kSpV + vs * kTileBytes, &tmV, &tmV32, BAR(S_V_FULL0 + vs),
+                                      pol_kv);
+                    ++nv;
+                }
+            }
+            for (uint32_t i = 1; i <= 2 && i <= nv; ++i) {
+                const uint32_t n = nv - i;
+                wait_bounded(BAR(S_V_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t kIdPV = idesc_bf16_f32(128, 128, false, true);
+            constexpr uint32_t kSlot = kTileBytes >> 4;  // descriptor step between ring slots
+            const uint64_t dQ0 = smem_desc(base + kSpQ, 16, 1024), dK0 = smem_desc(base + kSpK, 16, 1024);
+            const uint64_t dV0 = smem_desc(base + kSpV, kBoxBytes, 1024);
+            uint32_t nq = 0, n = 0, n_items = 0;
+            // the tile whose P V is still to be issued: sequence number, first / last tile of its item, item index
+            bool pend = false, pend_first = false, pend_last = false;
+            uint32_t pend_n = 0, pend_item = 0;
+            bool ok = true;
+            auto issue_pv = [&]() -> bool {
+                const uint32_t b = pend_n & 1u;
+                if (!wait_bounded(BAR(S_P_FULL0 + b), (pend_n >> 1) & 1u, lim)) return false;
+                if (!wait_bounded(BAR(S_V_FULL0 + b), (pend_n >> 1) & 1u, lim)) return false;
+                if (pend_first && pend_item > 0 && !wait_bounded(BAR(S_O_FREE), (pend_item - 1) & 1u, lim))
+                    return false;
+                tc_fence_after();
+                const uint64_t dV = dV0 + b * kSlot;
+#pragma unroll
+                for (uint32_t kk = 0; kk < 8; ++kk)
+                    tc_mma_ts(tO, tP + b * 64u + kk * 8u, dV + kk * 128u, kIdPV, (pend_first && kk == 0) ? 0u : 1u);
+                // the last tile's V slot is released by the epilogue, after it has staged O there
+                if (!pend_last) tc_commit(BAR(S_V_EMPTY0 + b));
+                tc_commit(BAR(S_PV_DONE0 + b));
+                pend = false;
+                return true;
+            };
+            SpItem it;
+            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
+                if (it.count <= 0) continue;
+                const uint32_t qs = nq & 1u;
+                if (!(ok = wait_bounded(BAR(S_Q_FULL0 + qs), (nq >> 1) & 1u, lim))) break;
+                ++nq;
+                // Q into TMEM buffer (item parity): 16 columns of Q per copy, in the A layout of the MMA. The buffer
+                // was last read by the previous item but one, whose MMAs completed before any S of the previous item
+                // was released. The copies run before this item's MMAs in the tensor pipe.
+                tc_fence_after();
+                const uint64_t dQ = dQ0 + qs * kSlot;
+                const uint32_t tQi = tQ + (n_items & 1u) * 64u;
+#pragma unroll
+                for (uint32_t kk = 0; kk < 8; ++kk)
+                    tc_cp_128x256b(tQi + kk * 8u, dQ + (((kk >> 2) * kBoxBytes + (kk & 3u) * 32u) >> 4));
+                tc_commit(BAR(S_Q_EMPTY0 + qs));  // the shared-memory Q slot is free once the copies are done
+                for (int t = 0; t < it.tiles; ++t, ++n) {
+                    const uint32_t ks = n % kSpKStages;
+                    if (!(ok = wait_bounded(BAR(S_K_FULL0 + ks), (n / kSpKStages) & 1u, lim))) break;
+                    // S is free once both softmax groups have read tile n - 1 from it
+                    if (n >= 1 && !(ok = wait_bounded(BAR(S_S_FREE), (n - 1) & 1u, lim))) break;
+                    tc_fence_after();
+                    const uint64_t dK = dK0 + ks * kSlot;
+#pragma unroll
+                    for (uint32_t kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3u) * 32u) >> 4;
+                        tc_mma_ts(tS, tQi + kk * 8u, dK + off, kIdQK, kk ? 1u : 0u);
+                    }
+                    tc_commit(BAR(S_S_FULL));
+                    tc_commit(BAR(S_K_EMPTY0 + ks));
+                    // the previous tile's P V goes behind this QK^T in the tensor pipe
+                    if (pend && !(ok = issue_pv())) break;
+                    pend = true;
+                    pend_first = (t == 0);
+                    pend_last = (t == it.tiles - 1);
+                    pend_n = n;
+                    pend_item = n_items;
+                }
+                ++n_items;
+            }
+            if (ok && pend) issue_pv();
+            tc_commit(BAR(S_MMA_DONE));
+            wait_bounded(BAR(S_MMA_DONE), 0, kDrainLimitNs);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // --------------------------------------------------------------------------- softmax warpgroups
+        const uint32_t grp = (uint32_t)(warp - 4) >> 2;  // keys 64 * grp .. 64 * grp + 63 of every tile
+        const uint32_t wl = (uint32_t)warp & 3u;
+        const int row = (int)(wl * 32u + lane);
+        const uint32_t lane_off = (wl * 32u) << 16;
+        const float c = a.scale_log2;
+        uint32_t n = 0, n_x = 0, n_items = 0;
+        bool ok = true;
+        SpItem it;
+        for (int r = 0; ok && (ok = next_item(r, it, true)) && !it.end; ++r) {
+            if (it.count <= 0) continue;
+            const size_t grow = (size_t)it.h * a.Np + it.qb * kTcRows + row;
+            float m_raw = -INFINITY, l_run = 0.0f;
+            uint32_t kvn = it.kv4;
+            for (int t = 0; t < it.tiles; ++t, ++n) {
+                const uint32_t kv4 = kvn;  // real keys per 32-column quarter of this tile
+                if (t + 1 < it.tiles) kvn = sp_quarter_keys<SUB>(a, it, t + 1);  // prefetched one tile ahead
+                const uint32_t kq0 = (kv4 >> (16 * grp)) & 255u, kq1 = (kv4 >> (16 * grp + 8)) & 255u;
+                const bool full = kq0 == 32u && kq1 == 32u;
+                const uint32_t b = n & 1u;
+                if (!(ok = wait_bounded_warp(BAR(S_S_FULL), n & 1u, lim))) break;
+                tc_fence_after();
+                float s[64];
+                tmem_ld32(tS + grp * 64u + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+                tmem_ld32(tS + grp * 64u + lane_off + 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(BAR(S_S_FREE));
+                if (!full) {  // keys past the sequence end, or quarters without a listed block, do not exist
+#pragma unroll
+                    for (int cc = 0; cc < 64; ++cc)
+                        if ((uint32_t)(cc & 31) >= (cc < 32 ? kq0 : kq1)) s[cc] = -INFINITY;
+                }
+                float tmax;
+                {
+                    float mx[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+#pragma unroll
+                    for (int cc = 24; cc < 64; cc += 16)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], s[cc + e], s[cc + 8 + e]);
+                    tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+                }
+                // The tile's row max over both groups' columns, exchanged through shared memory.
+                float* const xm = xmax + (n_x & 1u) * 256u;
+                xm[grp * 128u + row] = tmax;
+                mbar_arrive(BAR(S_MAX_X));
+                if (!(ok = wait_bounded_warp(BAR(S_MAX_X), n_x & 1u, lim))) break;
+                ++n_x;
+                tmax = fmaxf(tmax, xm[(grp ^ 1u) * 128u + row]);
+                // Reference max: raised only when the tile max exceeds it by more than 2^8 in the exp2 domain. A row
+                // that has seen no real key yet keeps a finite reference so that its weights are exact zeros.
+                const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
+                const float alpha = (t > 0 && need && tmax != -INFINITY) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
+                if (need) m_raw = (tmax == -INFINITY) ? (t == 0 ? 0.0f : m_raw) : tmax;
+                const float neg_mc = -m_raw * c;
+                uint32_t pw[32];
+                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                if (full) {
+                    // three pairs in eight on the FMA pipe (packed polynomial), the rest on the exp unit
+                    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
+                        float p0, p1;
+                        if ((e & 7) >= 5) {
+                            exp2_poly2(xx, p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(xx, x0, x1);
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        pw[e] = pack_bf16x2(p0, p1);
+                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float p0 = (s[2 * e] != -INFINITY) ? ex2_approx(fmaf(s[2 * e], c, neg_mc)) : 0.0f;
+                        const float p1 = (s[2 * e + 1] != -INFINITY) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_mc)) : 0.0f;
+                        pw[e] = pack_bf16x2(p0, p1);
+                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                    }
+                }
+                float la, lb, lc, ld;
+                f2_unpack(l2[0], la, lb);
+                f2_unpack(l2[1], lc, ld);
+                l_run = l_run * alpha + ((la + lb) + (lc + ld));
+                // O holds the sum up to tile n - 1 once that tile's P V has completed; this group rescales its 64
+                // columns before this tile's P V may add to them.
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    if (!(ok = wait_bounded_warp(BAR(S_PV_DONE0 + (b ^ 1u)), ((n - 1) >> 1) & 1u, lim))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + grp * 64u + lane_off + ch * 32u, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st32(tO + grp * 64u + lane_off + ch * 32u, ov);
+                    }
+                }
+                // P buffer b was last read by P V of tile n - 2, issued before QK^T of tile n; this tile's S was
+                // written after it completed.
+                tmem_st32(tP + b * 64u + grp * 32u + lane_off, pw);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(S_P_FULL0 + b));
+            }
+            if (!ok) break;
+            // Epilogue: full row sum from both groups, O / l for this group's 64 columns staged in the released V
+            // slot, one TMA store per group. The sums travel through the row-max buffer of the item's last tile:
+            // once the last P V is done, both groups have passed their reads of it (that P V needed both groups'
+            // P), and the next item's first tile uses the other buffer.
+            const uint32_t nl = n - 1;
+            if (!(ok = wait_bounded_warp(BAR(S_PV_DONE0 + (nl & 1u)), (nl >> 1) & 1u, lim))) break;
+            tc_fence_after();
+            float* const xsum = xmax + ((n_x - 1u) & 1u) * 256u;
+            xsum[grp * 128u + row] = l_run;
+            mbar_arrive(BAR(S_SUM_X));
+            if (!(ok = wait_bounded_warp(BAR(S_SUM_X), n_items & 1u, lim))) break;
+            const float l_all = l_run + xsum[(grp ^ 1u) * 128u + row];
+            const float inv_l = 1.0f / l_all;
+            uint32_t ov[2][32];
+            tmem_ld32(tO + grp * 64u + lane_off, ov[0]);
+            tmem_ld32(tO + grp * 64u + lane_off + 32u, ov[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(BAR(S_O_FREE));  // the next item's first P V may overwrite O
+            const uint32_t stage = base + kSpV + (nl & 1u) * kTileBytes + grp * kBoxBytes;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t j = (uint32_t)(ch * 4 + q4);  // 16-byte chunk of this row's 128 bytes
+                    uint32_t w[4];
+#pragma unroll
+                    for (int k2 = 0; k2 < 4; ++k2)
+                        w[k2] = pack_bf16x2(__uint_as_float(ov[ch][q4 * 8 + 2 * k2]) * inv_l,
+                                            __uint_as_float(ov[ch][q4 * 8 + 2 * k2 + 1]) * inv_l);
+                    st_shared_v4(stage + (uint32_t)row * 128u + ((j ^ ((uint32_t)row & 7u)) << 4), w[0], w[1], w[2],
+                                 w[3]);
+                }
+            fence_proxy_async_smem();
+            mbar_arrive(BAR(S_ST_READY0 + grp));
+            if (!(ok = wait_bounded_warp(BAR(S_ST_READY0 + grp), n_items & 1u, lim))) break;
+            if (row == 0) {
+                tma_store_2d(&tmO, stage, 64 * (int)grp, it.h * a.Np + it.qb * kTcRows);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                if (grp == 1) {
+                    mbar_arrive(BAR(S_ST_DONE));
+                } else if ((ok = wait_bounded(BAR(S_ST_DONE), n_items & 1u, lim))) {
+                    // both boxes have left the slot: hand it back to the V producer
+                    mbar_arrive(BAR(S_V_EMPTY0 + (nl & 1u)));
+                }
+            }
+            if (!(ok = __all_sync(0xffffffffu, ok))) break;
+            if (a.lse && grp == 0) a.lse[grow] = (m_raw * c + lg2_approx(l_all)) * 0.6931471805599453f;
+            ++n_items;
+        }
+        if (row == 0) bulk_wait_all();  // the O stores have landed before the CTA exits
+    }
+    // Teardown: every role has left its loop (normally or after a bounded wait ran out).
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace losa

@@ -22,6 +22,7 @@ constexpr unsigned int kDevErrBadData = 2u;
 #include "attn_f32.cuh"
 #include "attn_tc.cuh"
 #include "attn_dense.cuh"
+#include "attn_sparse.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
 
@@ -118,14 +119,14 @@ losa_status launch_dense_kernel(int grid, const CUtensorMap& tq, const CUtensorM
     return launch_status();
 }
 
-template <bool M, int SUB>
-losa_status launch_tc_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tk32, const CUtensorMap& tv32, const TcArgs& a, cudaStream_t stream) {
-    const uint32_t smem = tc_smem_bytes<M>();
-    if (cudaFuncSetAttribute(attn_tc_kernel<M, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+template <int SUB>
+losa_status launch_sparse_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& tk32, const CUtensorMap& tv32, const CUtensorMap& to,
+                                 const TcArgs& a, cudaStream_t stream) {
+    if (cudaFuncSetAttribute(attn_sparse_kernel<SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpSmem) !=
         cudaSuccess)
         return LOSA_ERR_CUDA;
-    attn_tc_kernel<M, SUB><<<grid, kTcThreads, smem, stream>>>(tq, tk, tv, tk32, tv32, a);
+    attn_sparse_kernel<SUB><<<grid, kSpThreads, kSpSmem, stream>>>(tq, tk, tv, tk32, tv32, to, a);
     return launch_status();
 }
 
@@ -170,13 +171,13 @@ losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const 
         return c32 ? launch_dense_kernel<false, 4>(dgrid, tq, tk, tv, a, stream)
                    : launch_dense_kernel<false, 1>(dgrid, tq, tk, tv, a, stream);
     }
-    const int want = (a.n_items + 1) / 2;  // two lanes per CTA
-    const int grid = want < sms ? (want > 0 ? want : 1) : sms;
-    if (with_mass)
-        return c32 ? launch_tc_kernel<true, 4>(grid, tq, tk, tv, tk32, tv32, a, stream)
-                   : launch_tc_kernel<true, 1>(grid, tq, tk, tv, tk32, tv32, a, stream);
-    return c32 ? launch_tc_kernel<false, 4>(grid, tq, tk, tv, tk32, tv32, a, stream)
-               : launch_tc_kernel<false, 1>(grid, tq, tk, tv, tk32, tv32, a, stream);
+    // retained lists: one persistent CTA per SM, one stream of items each; masses come from dense steps only
+    if (with_mass) return LOSA_ERR_UNSUPPORTED;
+    const int grid = a.n_items < sms ? (a.n_items > 0 ? a.n_items : 1) : sms;
+    CUtensorMap to;  // O rows leave through TMA stores of 64-column boxes
+    if (!make_tile_map(&to, o, rows)) return LOSA_ERR_CUDA;
+    return c32 ? launch_sparse_kernel<4>(grid, tq, tk, tv, tk32, tv32, to, a, stream)
+               : launch_sparse_kernel<1>(grid, tq, tk, tv, tk32, tv32, to, a, stream);
 }
 
 template <int D>
