@@ -259,8 +259,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int e = 0; e < 64; ++e) {
                         const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
                         float p0, p1;
-                        if ((e & 7) >= 5) {
-                            exp2_poly2(xx, p0, p1);
+                        if ((e & 3) == 3) {
+                            exp2_poly2_d3(xx, p0, p1);
                         } else {
                             float x0, x1;
                             f2_unpack(xx, x0, x1);

@@ -141,6 +141,27 @@ __device__ __forceinline__ void exp2_poly2(uint64_t xx, float& r0, float& r1) {
     r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// Degree-3 variant for the forward P, which is rounded to bf16 (relative step 2^-8) right after: coefficients fitted
+// the same way, max relative error 7.5e-5 in fp32 Horner form. One packed FMA fewer per pair than exp2_poly2.
+constexpr float kExp2D0 = 0.9999280571937561f, kExp2D1 = 0.6932609677314758f, kExp2D2 = 0.2426111251115799f,
+                kExp2D3 = 0.0551716685295105f;
+__device__ __forceinline__ void exp2_poly2_d3(uint64_t xx, float& r0, float& r1) {
+    float x0, x1;
+    f2_unpack(xx, x0, x1);
+    xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = f2_add(xx, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), xx);
+    uint64_t p = f2_fma(f2_pack(kExp2D3, kExp2D3), f, f2_pack(kExp2D2, kExp2D2));
+    p = f2_fma(p, f, f2_pack(kExp2D1, kExp2D1));
+    p = f2_fma(p, f, f2_pack(kExp2D0, kExp2D0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]^T: the A operand (P) is read from tensor memory.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
