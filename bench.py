@@ -177,11 +177,11 @@ def oracle_sample_run(cfg, qkv, tau, n_items, seed=7):
     q, k, v = qkv
     items = sample_items(cfg, n_items, seed=seed)[:n_items]
     scale = 1.0 / math.sqrt(cfg.head_dim)
-    R, N = cfg.block, cfg.n_tokens
+    R, C, N = cfg.block, cfg.kblock, cfg.n_tokens
     t0 = time.perf_counter()
     oracle.dense(q, k, v, N, R, scale, items)
     t1 = time.perf_counter()
-    m = oracle.mass(q, k, N, R, R, scale, items)
+    m = oracle.mass(q, k, N, R, C, scale, items)
     t2 = time.perf_counter()
     counts, idx = oracle.select(m.astype(np.float32), tau)
     t3 = time.perf_counter()
@@ -193,11 +193,11 @@ def oracle_sample_run(cfg, qkv, tau, n_items, seed=7):
     indptr[1:] = np.cumsum(full_counts)
     kv = np.concatenate([idx[t, :counts[t]] for t in range(len(items))]).astype(np.int32)
     t4 = time.perf_counter()
-    oracle.sparse(q, k, v, N, R, R, scale, indptr, kv, items)
+    oracle.sparse(q, k, v, N, R, C, scale, indptr, kv, items)
     t5 = time.perf_counter()
     n = len(items)
     return {"items": n, "dense_s": (t1 - t0) / n, "mass_s": (t2 - t1) / n, "select_s": (t3 - t2) / n,
-            "sparse_s": (t5 - t4) / n, "density": float(counts.sum()) / (n * cfg.n_blocks),
+            "sparse_s": (t5 - t4) / n, "density": float(counts.sum()) / (n * cfg.n_kblocks),
             "threads": oracle.num_threads()}
 
 
@@ -247,31 +247,58 @@ def run_reference(args, cfg):
 
 # ---------------------------------------------------------------------------------------------- native path
 
+class RankGroup:
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK from the launcher): barriers around the timed region and
+    the max over ranks of each device-timed duration. Every rank takes the same collective steps in the same order."""
+
+    def __init__(self, backend="nccl", timeout_s=600):
+        import torch
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x):
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def whole_job_value(world, steps, flop_per_step, seconds_max):
+    """Whole-job throughput in TFLOP/s: every rank runs `steps` steps of `flop_per_step` (weak scaling), the job
+    takes as long as its slowest rank."""
+    return world * steps * flop_per_step / seconds_max / 1e12
+
+
 def run_native(args, cfg):
     import torch
     import free_block_sparse_losa_b200 as L
     from free_block_sparse_losa_b200.harness import LayerBuffers, host_tokens_to_device
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    group = RankGroup("nccl")
+    rank, world, local = group.rank, group.world, group.local
+    barrier, max_over_ranks = group.barrier, group.max
 
     L.load()
     layer = make_layer(cfg)
@@ -321,7 +348,7 @@ def run_native(args, cfg):
 
     work = work_model(cfg, nnz)
     K = args.steps
-    value = world * K * work["dense_equiv_flop"] / t_sparse / 1e12
+    value = whole_job_value(world, K, work["dense_equiv_flop"], t_sparse)
 
     # end to end through the C ABI with host buffers: pinned Q/K/V -> device, sparse attention, O -> pinned host
     e2e = None
@@ -353,7 +380,7 @@ def run_native(args, cfg):
             raise RuntimeError("device error in the end-to-end loop")
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
         d2h = ho.numel() * ho.element_size()
-        e2e = {"value": round(world * K * work["dense_equiv_flop"] / t_e2e / 1e12, 3),
+        e2e = {"value": round(whole_job_value(world, K, work["dense_equiv_flop"], t_e2e), 3),
                "unit": "TFLOP/s (dense-equivalent, sparse attention incl. host copies)",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_call": round(t_e2e / K * 1e3, 3)}
 
@@ -384,11 +411,11 @@ def run_native(args, cfg):
     per_sel = t_sel / K
     tr = measured_traffic(cfg.name)
     roof = {
-        "dense_profile": roofline("attn_tc_kernel<1> (losa_dense_profile: dense forward + block masses)", "tensor",
+        "dense_profile": roofline("attn_dense_kernel<1> (losa_dense_profile: dense forward + block masses)", "tensor",
                                   work["profile_flop"], per_prof, pk, "TFLOP/s", tr.get("dense_profile")),
         "select": roofline("select_rows + select_finalize + select_scatter (losa_select)", "hbm",
                            work["select_bytes"], per_sel, pk, "GB/s", tr.get("select")),
-        "sparse_attn": roofline("attn_tc_kernel<0> over the retained lists (losa_sparse_attn)", "tensor",
+        "sparse_attn": roofline("attn_sparse_kernel over the retained lists (losa_sparse_attn)", "tensor",
                                 work["sparse_flop"], per_sparse, pk, "TFLOP/s", tr.get("sparse_attn")),
     }
     dominant = max(("dense_profile", per_prof), ("select", per_sel), ("sparse_attn", per_sparse),
@@ -426,9 +453,7 @@ def run_native(args, cfg):
                                         f"{cfg.heads * cfg.n_blocks} items")
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    group.close()
     return 0
 
 
