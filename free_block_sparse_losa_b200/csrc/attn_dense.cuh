@@ -13,8 +13,8 @@
 //   t). They exchange their half-tile row maxima through shared memory, apply the same running max, keep their own
 //   partial row sums, rescale their own half of O, and write their own half of P. P V runs as two groups of eight
 //   N = 128 instructions (keys 0..127 and 128..255) with P read from TMEM and V from shared memory (MN-major).
-//   Warp 0 issues TMA (Q once per item; K single-buffered, V double-buffered, 64 KB per 256-key tile), warp 1 issues
-//   the MMAs and owns TMEM.
+//   Warp 0 issues the TMA loads of Q (once per item) and K (single-buffered), warp 2 those of V (double-buffered),
+//   64 KB per 256-key tile; each box of a tile comes from its own lane. Warp 1 issues the MMAs and owns TMEM.
 //   Mass phase (same item, Q still in shared memory, lse exact in registers): S is recomputed for every 256-key tile
 //   and each warpgroup sums 2^(s*c - lse2) over its 128 columns per key block; per-warp partials go to the idle V
 //   buffer and are flushed to M every 1024 blocks.
@@ -35,7 +35,7 @@ constexpr uint32_t kDnSmem = kDnXchg + 2 * 2 * 128 * 4;  // 231680 bytes: needs 
 
 enum : uint32_t {
     D_Q_FULL = 0, D_Q_EMPTY, D_K_FULL, D_K_EMPTY, D_V_FULL0, D_V_FULL1, D_V_EMPTY0, D_V_EMPTY1, D_S_FULL, D_S_FREE,
-    D_P_FULL, D_PV_DONE, D_O_FREE, D_MAX_X, D_SUM_X, D_PART, D_PART2, D_MMA_DONE, D_COUNT
+    D_P_FULL, D_PV_DONE, D_O_FREE, D_MAX_X, D_SUM_X, D_PART, D_PART2, D_MASS_DONE, D_MMA_DONE, D_COUNT
 };
 
 template <bool WITH_MASS, int SUB>
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < D_COUNT; ++s) {
             const bool wide = s == D_S_FREE || s == D_P_FULL || s == D_O_FREE || s == D_MAX_X || s == D_SUM_X ||
-                              s == D_PART || s == D_PART2;
+                              s == D_PART || s == D_PART2 || s == D_MASS_DONE;
             mbar_init(BAR(s), wide ? 256u : 1u);
         }
         fence_barrier_init();
@@ -85,58 +85,64 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int G = gridDim.x;
 
     if (warp == 0) {
-        // ------------------------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            const uint64_t pol_q = l2_policy_evict_first();
-            const uint64_t pol_kv = l2_policy_evict_last();
-            uint32_t nq = 0, nk_ld = 0, nv_ld = 0;
-            bool ok = true;
-            for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
-                const int h = w / a.nq, qb = w - h * a.nq;
-                if (!(ok = wait_bounded(BAR(D_Q_EMPTY), (nq & 1u) ^ 1u, lim))) break;
-                const int32_t qrow = h * a.Np + qb * kTcRows;
-                mbar_arrive_expect_tx(BAR(D_Q_FULL), kTileBytes);
-                tma_load_2d_hint(base + kDnQ, &tmQ, 0, qrow, BAR(D_Q_FULL), pol_q);
-                tma_load_2d_hint(base + kDnQ + kBoxBytes, &tmQ, 64, qrow, BAR(D_Q_FULL), pol_q);
-                ++nq;
-                for (int t = 0; t < T + mass_tiles; ++t) {
-                    const bool fwd = t < T;
-                    const int32_t krow = h * a.Np + (fwd ? t : t - T) * 256;  // rows past the head are masked
-                    if (!(ok = wait_bounded(BAR(D_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
-                    mbar_arrive_expect_tx(BAR(D_K_FULL), 2 * kTileBytes);
-#pragma unroll
-                    for (int dh = 0; dh < 2; ++dh)
-#pragma unroll
-                        for (int rh = 0; rh < 2; ++rh)
-                            tma_load_2d_hint(base + kDnK + dh * 32768u + rh * 16384u, &tmK, 64 * dh, krow + 128 * rh,
-                                             BAR(D_K_FULL), pol_kv);
-                    ++nk_ld;
-                    if (fwd) {
-                        const uint32_t vb = nv_ld & 1u;
-                        if (!(ok = wait_bounded(BAR(D_V_EMPTY0 + vb), ((nv_ld >> 1) & 1u) ^ 1u, lim))) break;
-                        mbar_arrive_expect_tx(BAR(D_V_FULL0 + vb), 2 * kTileBytes);
-#pragma unroll
-                        for (int dh = 0; dh < 2; ++dh)
-#pragma unroll
-                            for (int rh = 0; rh < 2; ++rh)
-                                tma_load_2d_hint(base + kDnV + vb * 65536u + dh * 32768u + rh * 16384u, &tmV, 64 * dh,
-                                                 krow + 128 * rh, BAR(D_V_FULL0 + vb), pol_kv);
-                        ++nv_ld;
-                    }
-                }
-                // The mass phase reuses V buffer 0 for partial sums: before loading the next item's V, wait until the
-                // softmax has flushed this item's last chunk (PART2 completes once per chunk).
-                if (WITH_MASS && ok) {
-                    const uint32_t chunks = (uint32_t)((T * 2 * SUB + kMaxMassBlocks - 1) / kMaxMassBlocks);
-                    if (!(ok = wait_bounded(BAR(D_PART2), (nq * chunks - 1u) & 1u, lim))) break;
-                }
+        // ------------------------------------------------------------- TMA producer: Q and K (whole warp)
+        // Every 16 KB box of a tile is issued by its own lane (lane 0 posts the expected bytes first): one thread's
+        // TMA loads are served one after another at about 30 bytes per clock, too slow for 64 KB per tile.
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const uint32_t dh = lane >> 1, rh = lane & 1u;  // box of lane < 4: column half dh, row half rh
+        uint32_t nq = 0, nk_ld = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
+            const int h = w / a.nq, qb = w - h * a.nq;
+            if (!(ok = wait_bounded_warp(BAR(D_Q_EMPTY), (nq & 1u) ^ 1u, lim))) break;
+            const int32_t qrow = h * a.Np + qb * kTcRows;
+            if (lane == 0) mbar_arrive_expect_tx(BAR(D_Q_FULL), kTileBytes);
+            __syncwarp();
+            if (lane < 2) tma_load_2d_hint(base + kDnQ + lane * kBoxBytes, &tmQ, 64 * (int)lane, qrow, BAR(D_Q_FULL), pol_q);
+            ++nq;
+            for (int t = 0; t < T + mass_tiles; ++t) {
+                const int32_t krow = h * a.Np + (t < T ? t : t - T) * 256;  // rows past the head are masked
+                if (!(ok = wait_bounded_warp(BAR(D_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
+                if (lane == 0) mbar_arrive_expect_tx(BAR(D_K_FULL), 2 * kTileBytes);
+                __syncwarp();
+                if (lane < 4)
+                    tma_load_2d_hint(base + kDnK + dh * 32768u + rh * 16384u, &tmK, 64 * (int)dh, krow + 128 * (int)rh,
+                                     BAR(D_K_FULL), pol_kv);
+                ++nk_ld;
             }
-            if (nq) wait_bounded(BAR(D_Q_FULL), (nq - 1) & 1u, kDrainLimitNs);
-            if (nk_ld) wait_bounded(BAR(D_K_FULL), (nk_ld - 1) & 1u, kDrainLimitNs);
-            for (uint32_t vb = 0; vb < 2; ++vb) {
-                const uint32_t n = (nv_ld + 1u - vb) >> 1;
-                if (n) wait_bounded(BAR(D_V_FULL0 + vb), (n - 1) & 1u, kDrainLimitNs);
+        }
+        if (nq) wait_bounded(BAR(D_Q_FULL), (nq - 1) & 1u, kDrainLimitNs);
+        if (nk_ld) wait_bounded(BAR(D_K_FULL), (nk_ld - 1) & 1u, kDrainLimitNs);
+        __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------------------------- TMA producer: V (whole warp)
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const uint32_t dh = lane >> 1, rh = lane & 1u;
+        uint32_t nv_ld = 0, n_it = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
+            const int h = w / a.nq;
+            for (int t = 0; t < T; ++t) {
+                const int32_t krow = h * a.Np + t * 256;
+                const uint32_t vb = nv_ld & 1u;
+                if (!(ok = wait_bounded_warp(BAR(D_V_EMPTY0 + vb), ((nv_ld >> 1) & 1u) ^ 1u, lim))) break;
+                if (lane == 0) mbar_arrive_expect_tx(BAR(D_V_FULL0 + vb), 2 * kTileBytes);
+                __syncwarp();
+                if (lane < 4)
+                    tma_load_2d_hint(base + kDnV + vb * 65536u + dh * 32768u + rh * 16384u, &tmV, 64 * (int)dh,
+                                     krow + 128 * (int)rh, BAR(D_V_FULL0 + vb), pol_kv);
+                ++nv_ld;
             }
+            // The mass phase reuses V buffer 0 for partial sums: before loading the next item's V, wait until the
+            // softmax has flushed this item's last chunk. MASS_DONE completes once per item, so its phase cannot be
+            // confused with a later one: the next item's needs this warp's next V loads.
+            if (WITH_MASS && ok && !(ok = wait_bounded_warp(BAR(D_MASS_DONE), n_it & 1u, lim))) break;
+            ++n_it;
+        }
+        for (uint32_t vb = 0; vb < 2; ++vb) {
+            const uint32_t n = (nv_ld + 1u - vb) >> 1;
+            if (n) wait_bounded(BAR(D_V_FULL0 + vb), (n - 1) & 1u, kDrainLimitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -429,6 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ++n_chunks;
                 }
                 if (!ok) break;
+                mbar_arrive(BAR(D_MASS_DONE));  // every chunk of this item is flushed: V buffer 0 is free again
             }
             ++n_items;
         }

@@ -13,6 +13,8 @@
 //            role waits on dependent global loads at an item boundary.
 //   warp 0   TMA: Q double-buffered (the next item's Q arrives during this item), K in a three-stage ring.
 //   warp 2   TMA: V in a two-stage ring (a V slot waiting for its P V never holds back K).
+//            In both producer warps every TMA box of a tile is issued by its own lane: one thread's TMA loads are
+//            served one after another at about 30 bytes per clock, which would cap a 32 KB tile at ~1100 clocks.
 //   warp 1   MMA: at an item's start, Q is copied from shared memory into TMEM (tcgen05.cp); then per tile
 //            S_n = Q K^T (128 x 128, N = 128, Q read from TMEM) and O += P V of tile n - 1 (P from TMEM). With both
 //            A operands in TMEM, the MMAs read only K and V from shared memory.
@@ -66,24 +68,25 @@ __device__ __forceinline__ int sp_block(const TcArgs& a, const SpItem& it, int e
     return (j < 0) ? 0 : (j >= a.nkb ? a.nkb - 1 : j);
 }
 
+// Loads tile t of an item into dst, one 16 KB (C = 128) or 4 KB (C = 32) box per lane; lane 0 posts the expected
+// bytes first. Called by all lanes of the producer warp.
 template <int SUB>
 __device__ __forceinline__ void sp_load_tile(const TcArgs& a, const SpItem& it, int t, uint32_t dst,
                                              const CUtensorMap* tm, const CUtensorMap* tm32, uint32_t bar,
-                                             uint64_t pol) {
-    mbar_arrive_expect_tx(bar, kTileBytes);
+                                             uint64_t pol, uint32_t lane) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
+    __syncwarp();
     if (SUB == 1) {
-        const int32_t krow = it.h * a.Np + sp_block(a, it, t) * kTcRows;
-        tma_load_2d_hint(dst, tm, 0, krow, bar, pol);
-        tma_load_2d_hint(dst + kBoxBytes, tm, 64, krow, bar, pol);
-    } else {
-#pragma unroll
-        for (int g = 0; g < SUB; ++g) {
-            // a missing quarter reloads the tile's first block (finite data, masked to P = 0)
-            const int e = SUB * t + g < it.count ? SUB * t + g : SUB * t;
-            const int32_t r32 = it.h * a.Np + sp_block(a, it, e) * 32;
-            tma_load_2d_hint(dst + g * 4096u, tm32, 0, r32, bar, pol);
-            tma_load_2d_hint(dst + kBoxBytes + g * 4096u, tm32, 64, r32, bar, pol);
+        if (lane < 2) {
+            const int32_t krow = it.h * a.Np + sp_block(a, it, t) * kTcRows;
+            tma_load_2d_hint(dst + lane * kBoxBytes, tm, 64 * (int)lane, krow, bar, pol);
         }
+    } else if (lane < 2 * SUB) {
+        const int g = (int)(lane >> 1), hx = (int)(lane & 1u);
+        // a missing quarter reloads the tile's first block (finite data, masked to P = 0)
+        const int e = SUB * t + g < it.count ? SUB * t + g : SUB * t;
+        const int32_t r32 = it.h * a.Np + sp_block(a, it, e) * 32;
+        tma_load_2d_hint(dst + hx * kBoxBytes + g * 4096u, tm32, 64 * hx, r32, bar, pol);
     }
 }
 
@@ -161,12 +164,13 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     const uint32_t tS = tmem, tO = tmem + 128u, tP = tmem + 256u, tQ = tmem + 384u;
     const unsigned long long lim = a.wait_limit_ns;
 
-    // Item record of round r from the ring (false on a timeout); every consumer thread arrives on its slot.
-    auto next_item = [&](int r, SpItem& it, bool warp_wide) -> bool {
+    // Item record of round r from the ring (false on a timeout). mode 0: one thread waits and arrives; 1: the whole
+    // warp waits and every lane arrives; 2: the whole warp waits and lane 0 arrives for it.
+    auto next_item = [&](int r, SpItem& it, int mode) -> bool {
         const uint32_t sl = (uint32_t)r & (kSpRingSlots - 1);
         const uint32_t par = ((uint32_t)r / kSpRingSlots) & 1u;
-        const bool ok = warp_wide ? wait_bounded_warp(BAR(S_IT_FULL0 + sl), par, lim)
-                                  : wait_bounded(BAR(S_IT_FULL0 + sl), par, lim);
+        const bool ok = mode ? wait_bounded_warp(BAR(S_IT_FULL0 + sl), par, lim)
+                             : wait_bounded(BAR(S_IT_FULL0 + sl), par, lim);
         if (!ok) return false;
         const volatile SpItem* src = &ring[sl];
         it.id = src->id;
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         it.tiles = src->tiles;
         it.kv4 = src->kv4;
         it.end = src->end;
-        mbar_arrive(BAR(S_IT_EMPTY0 + sl));
+        if (mode != 2 || lane == 0) mbar_arrive(BAR(S_IT_EMPTY0 + sl));
         return true;
     };
 
@@ -223,62 +227,59 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         __syncwarp();
     } else if (warp == 0) {
-        // ----------------------------------------------------------------------------- TMA producer: Q and K
-        if (lane == 0) {
-            const uint64_t pol_q = l2_policy_evict_first();
-            const uint64_t pol_kv = l2_policy_evict_last();
-            uint32_t nq = 0, nk = 0;
-            bool ok = true;
-            SpItem it;
-            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
-                if (it.count <= 0) continue;
-                const uint32_t qs = nq & 1u;
-                if (!(ok = wait_bounded(BAR(S_Q_EMPTY0 + qs), ((nq >> 1) & 1u) ^ 1u, lim))) break;
-                const int32_t qrow = it.h * a.Np + it.qb * kTcRows;
-                mbar_arrive_expect_tx(BAR(S_Q_FULL0 + qs), kTileBytes);
-                tma_load_2d_hint(base + kSpQ + qs * kTileBytes, &tmQ, 0, qrow, BAR(S_Q_FULL0 + qs), pol_q);
-                tma_load_2d_hint(base + kSpQ + qs * kTileBytes + kBoxBytes, &tmQ, 64, qrow, BAR(S_Q_FULL0 + qs),
-                                 pol_q);
-                ++nq;
-                for (int t = 0; t < it.tiles; ++t) {
-                    const uint32_t ks = nk % kSpKStages;
-                    if (!(ok = wait_bounded(BAR(S_K_EMPTY0 + ks), ((nk / kSpKStages) & 1u) ^ 1u, lim))) break;
-                    sp_load_tile<SUB>(a, it, t, base + kSpK + ks * kTileBytes, &tmK, &tmK32, BAR(S_K_FULL0 + ks),
-                                      pol_kv);
-                    ++nk;
-                }
+        // ----------------------------------------------------------------- TMA producer: Q and K (whole warp)
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        uint32_t nq = 0, nk = 0;
+        bool ok = true;
+        SpItem it;
+        for (int r = 0; ok && (ok = next_item(r, it, 2)) && !it.end; ++r) {
+            if (it.count <= 0) continue;
+            const uint32_t qs = nq & 1u;
+            if (!(ok = wait_bounded_warp(BAR(S_Q_EMPTY0 + qs), ((nq >> 1) & 1u) ^ 1u, lim))) break;
+            const int32_t qrow = it.h * a.Np + it.qb * kTcRows;
+            if (lane == 0) mbar_arrive_expect_tx(BAR(S_Q_FULL0 + qs), kTileBytes);
+            __syncwarp();
+            if (lane < 2)
+                tma_load_2d_hint(base + kSpQ + qs * kTileBytes + lane * kBoxBytes, &tmQ, 64 * (int)lane, qrow,
+                                 BAR(S_Q_FULL0 + qs), pol_q);
+            ++nq;
+            for (int t = 0; t < it.tiles; ++t) {
+                const uint32_t ks = nk % kSpKStages;
+                if (!(ok = wait_bounded_warp(BAR(S_K_EMPTY0 + ks), ((nk / kSpKStages) & 1u) ^ 1u, lim))) break;
+                sp_load_tile<SUB>(a, it, t, base + kSpK + ks * kTileBytes, &tmK, &tmK32, BAR(S_K_FULL0 + ks), pol_kv,
+                                  lane);
+                ++nk;
             }
-            for (uint32_t i = 1; i <= 2 && i <= nq; ++i) {
-                const uint32_t n = nq - i;
-                wait_bounded(BAR(S_Q_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
-            }
-            for (uint32_t i = 1; i <= kSpKStages && i <= nk; ++i) {
-                const uint32_t n = nk - i;
-                wait_bounded(BAR(S_K_FULL0 + n % kSpKStages), (n / kSpKStages) & 1u, kDrainLimitNs);
-            }
+        }
+        for (uint32_t i = 1; i <= 2 && i <= nq; ++i) {
+            const uint32_t n = nq - i;
+            wait_bounded(BAR(S_Q_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
+        }
+        for (uint32_t i = 1; i <= kSpKStages && i <= nk; ++i) {
+            const uint32_t n = nk - i;
+            wait_bounded(BAR(S_K_FULL0 + n % kSpKStages), (n / kSpKStages) & 1u, kDrainLimitNs);
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ----------------------------------------------------------------------------------- TMA producer: V
-        if (lane == 0) {
-            const uint64_t pol_kv = l2_policy_evict_last();
-            uint32_t nv = 0;
-            bool ok = true;
-            SpItem it;
-            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
-                if (it.count <= 0) continue;
-                for (int t = 0; t < it.tiles; ++t) {
-                    const uint32_t vs = nv & 1u;
-                    if (!(ok = wait_bounded(BAR(S_V_EMPTY0 + vs), ((nv >> 1) & 1u) ^ 1u, lim))) break;
-                    sp_load_tile<SUB>(a, it, t, base + kSpV + vs * kTileBytes, &tmV, &tmV32, BAR(S_V_FULL0 + vs),
-                                      pol_kv);
-                    ++nv;
-                }
+        // --------------------------------------------------------------------------- TMA producer: V (whole warp)
+        const uint64_t pol_kv = l2_policy_evict_last();
+        uint32_t nv = 0;
+        bool ok = true;
+        SpItem it;
+        for (int r = 0; ok && (ok = next_item(r, it, 2)) && !it.end; ++r) {
+            if (it.count <= 0) continue;
+            for (int t = 0; t < it.tiles; ++t) {
+                const uint32_t vs = nv & 1u;
+                if (!(ok = wait_bounded_warp(BAR(S_V_EMPTY0 + vs), ((nv >> 1) & 1u) ^ 1u, lim))) break;
+                sp_load_tile<SUB>(a, it, t, base + kSpV + vs * kTileBytes, &tmV, &tmV32, BAR(S_V_FULL0 + vs), pol_kv,
+                                  lane);
+                ++nv;
             }
-            for (uint32_t i = 1; i <= 2 && i <= nv; ++i) {
-                const uint32_t n = nv - i;
-                wait_bounded(BAR(S_V_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
-            }
+        }
+        for (uint32_t i = 1; i <= 2 && i <= nv; ++i) {
+            const uint32_t n = nv - i;
+            wait_bounded(BAR(S_V_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 return true;
             };
             SpItem it;
-            for (int r = 0; ok && (ok = next_item(r, it, false)) && !it.end; ++r) {
+            for (int r = 0; ok && (ok = next_item(r, it, 0)) && !it.end; ++r) {
                 if (it.count <= 0) continue;
                 const uint32_t qs = nq & 1u;
                 if (!(ok = wait_bounded(BAR(S_Q_FULL0 + qs), (nq >> 1) & 1u, lim))) break;
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         uint32_t n = 0, n_x = 0, n_items = 0;
         bool ok = true;
         SpItem it;
-        for (int r = 0; ok && (ok = next_item(r, it, true)) && !it.end; ++r) {
+        for (int r = 0; ok && (ok = next_item(r, it, 1)) && !it.end; ++r) {
             if (it.count <= 0) continue;
             const size_t grow = (size_t)it.h * a.Np + it.qb * kTcRows + row;
             float m_raw = -INFINITY, l_run = 0.0f;
