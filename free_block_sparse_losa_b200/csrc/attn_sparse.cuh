@@ -12,7 +12,7 @@
 //            memory (head, query block, list start and length, tiles, key validity of the first tile), so that no
 //            role waits on dependent global loads at an item boundary.
 //   warp 0   TMA: Q double-buffered (the next item's Q arrives during this item), K in a three-stage ring.
-//   warp 2   TMA: V in a two-stage ring (a V slot waiting for its P V never holds back K).
+//   warp 2   TMA: V in a two-stage ring (a V slot waiting for its P V never holds back K), and the O stores.
 //            In both producer warps every TMA box of a tile is issued by its own lane: one thread's TMA loads are
 //            served one after another at about 30 bytes per clock, which would cap a 32 KB tile at ~1100 clocks.
 //   warp 1   MMA: at an item's start, Q is copied from shared memory into TMEM (tcgen05.cp); then per tile
@@ -26,9 +26,11 @@
 // pairs, one buffer per item parity). O is rescaled in place only when a row's running max grows by more than 2^8
 // (the final division by the sum taken against the same reference keeps this exact); each group rescales its own 64
 // columns of O.
-// Epilogue: O / l in bf16 is written, 128-byte swizzled, into the V slot the item's last P V has just released and
-// leaves through two TMA stores (one 64-column box per group); the V producer gets the slot back once the stores
-// have read it. Row stores from registers would put 32 rows into every warp-wide store.
+// Epilogue, deferred until the next item's first tile is done (by then the item's last P V has completed): the two
+// groups add their partial row sums through TMEM (the first column of each group's half of the released P buffer),
+// write O / l in bf16, 128-byte swizzled, into the V slot the item's last P V has released, and go on. The V
+// producer stores the two 64-column boxes with TMA before it refills that slot. Row stores from registers would put
+// 32 rows into every warp-wide store; waiting for the TMA store would stall the softmax warps.
 // Every wait is bounded in time (LOSA_ERR_TIMEOUT in the device error word, then a clean exit).
 #pragma once
 #include <cstdint>
@@ -49,8 +51,8 @@ constexpr uint32_t kSpRingSlots = 4;
 
 enum : uint32_t {
     S_Q_FULL0 = 0, S_Q_EMPTY0 = 2, S_K_FULL0 = 4, S_K_EMPTY0 = 7, S_V_FULL0 = 10, S_V_EMPTY0 = 12, S_S_FULL = 14,
-    S_S_FREE = 16, S_P_FULL0 = 18, S_PV_DONE0 = 20, S_MAX_X = 22, S_SUM_X, S_O_FREE, S_ST_READY0, S_ST_READY1 = 26,
-    S_ST_DONE, S_IT_FULL0, S_IT_EMPTY0 = S_IT_FULL0 + kSpRingSlots, S_MMA_DONE = S_IT_EMPTY0 + kSpRingSlots, S_COUNT
+    S_S_FREE = 16, S_P_FULL0 = 18, S_PV_DONE0 = 20, S_MAX_X = 22, S_SUM_X, S_O_FREE, S_STAGED0, S_IT_FULL0 = S_STAGED0 + 2,
+    S_IT_EMPTY0 = S_IT_FULL0 + kSpRingSlots, S_MMA_DONE = S_IT_EMPTY0 + kSpRingSlots, S_COUNT
 };
 constexpr int kSpThreads = 384;  // 12 warps: 0 Q/K TMA, 1 MMA, 2 V TMA, 3 work order, 4..11 softmax
 static_assert(S_COUNT <= 47, "barrier slots");
@@ -132,11 +134,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < S_COUNT; ++s) {
             uint32_t cnt = 1;
-            if (s == S_S_FREE || s == S_P_FULL0 || s == S_P_FULL0 + 1 || s == S_MAX_X ||
-                s == S_SUM_X || s == S_O_FREE)
+            if (s == S_S_FREE || s == S_P_FULL0 || s == S_P_FULL0 + 1 || s == S_MAX_X || s == S_SUM_X ||
+                s == S_O_FREE || s == S_STAGED0 || s == S_STAGED0 + 1)
                 cnt = 256;
-            else if (s == S_ST_READY0 || s == S_ST_READY1)
-                cnt = 128;
             else if (s >= S_IT_EMPTY0 && s < S_IT_EMPTY0 + kSpRingSlots)
                 cnt = 3 + 256;  // Q/K producer, V producer, MMA issuer, 256 softmax threads
             mbar_init(BAR(s), cnt);
@@ -262,21 +262,54 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         __syncwarp();
     } else if (warp == 2) {
-        // --------------------------------------------------------------------------- TMA producer: V (whole warp)
+        // ------------------------------------------------------------- TMA producer: V and the O stores (whole warp)
+        // A V slot whose last tile closed an item holds that item's staged O when it is wanted again: its two
+        // 64-column boxes are stored (one lane each) and read out before the slot is refilled. Other slots come back
+        // through V_EMPTY from the MMA.
         const uint64_t pol_kv = l2_policy_evict_last();
         uint32_t nv = 0;
+        uint32_t empty_cnt[2] = {0u, 0u}, staged_cnt[2] = {0u, 0u};
+        bool fin[2] = {false, false};
+        int32_t fin_row[2] = {0, 0};
         bool ok = true;
+        auto flush = [&](uint32_t sl) -> bool {
+            if (!wait_bounded_warp(BAR(S_STAGED0 + sl), staged_cnt[sl] & 1u, lim)) return false;
+            ++staged_cnt[sl];
+            if (lane < 2) {
+                tma_store_2d(&tmO, base + kSpV + sl * kTileBytes + lane * kBoxBytes, 64 * (int)lane, fin_row[sl]);
+                bulk_commit_group();
+                bulk_wait_read_all();
+            }
+            __syncwarp();
+            fin[sl] = false;
+            return true;
+        };
         SpItem it;
         for (int r = 0; ok && (ok = next_item(r, it, 2)) && !it.end; ++r) {
             if (it.count <= 0) continue;
             for (int t = 0; t < it.tiles; ++t) {
                 const uint32_t vs = nv & 1u;
-                if (!(ok = wait_bounded_warp(BAR(S_V_EMPTY0 + vs), ((nv >> 1) & 1u) ^ 1u, lim))) break;
+                if (nv >= 2) {
+                    if (fin[vs]) {
+                        if (!(ok = flush(vs))) break;
+                    } else {
+                        if (!(ok = wait_bounded_warp(BAR(S_V_EMPTY0 + vs), empty_cnt[vs] & 1u, lim))) break;
+                        ++empty_cnt[vs];
+                    }
+                }
                 sp_load_tile<SUB>(a, it, t, base + kSpV + vs * kTileBytes, &tmV, &tmV32, BAR(S_V_FULL0 + vs), pol_kv,
                                   lane);
+                fin[vs] = (t == it.tiles - 1);
+                fin_row[vs] = it.h * a.Np + it.qb * kTcRows;
                 ++nv;
             }
         }
+        // the last one or two items' O, oldest slot first
+        for (uint32_t k = 0; ok && k < 2; ++k) {
+            const uint32_t sl = (nv + k) & 1u;
+            if (fin[sl]) ok = flush(sl);
+        }
+        if (lane < 2) bulk_wait_all();  // the O stores have landed before the CTA exits
         for (uint32_t i = 1; i <= 2 && i <= nv; ++i) {
             const uint32_t n = nv - i;
             wait_bounded(BAR(S_V_FULL0 + (n & 1u)), (n >> 1) & 1u, kDrainLimitNs);
@@ -364,8 +397,57 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         const int row = (int)(wl * 32u + lane);
         const uint32_t lane_off = (wl * 32u) << 16;
         const float c = a.scale_log2;
-        uint32_t n = 0, n_x = 0, n_items = 0;
+        uint32_t n = 0, n_x = 0, n_epi = 0;
         bool ok = true;
+        // An item's epilogue waits until the next item's first tile is done: by then the item's last P V has
+        // completed, where an immediate epilogue would sit waiting for it.
+        bool pend = false;
+        size_t pd_grow = 0;
+        float pd_m = 0.0f, pd_l = 0.0f;
+        uint32_t pd_nl = 0;
+        auto epilogue = [&]() -> bool {
+            const uint32_t bl = pd_nl & 1u;
+            if (!wait_bounded_warp(BAR(S_PV_DONE0 + bl), (pd_nl >> 1) & 1u, lim)) return false;
+            tc_fence_after();
+            // Full row sum: each group puts its partial sum into the first column of its half of the P buffer that
+            // the item's last P V has just released (rewritten only by tile pd_nl + 2, after both groups' next max
+            // exchange).
+            const uint32_t tsum = tP + bl * 64u + lane_off;
+            tmem_st1(tsum + grp * 32u, __float_as_uint(pd_l));
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(S_SUM_X));
+            if (!wait_bounded_warp(BAR(S_SUM_X), n_epi & 1u, lim)) return false;
+            tc_fence_after();
+            const float l_all = pd_l + __uint_as_float(tmem_ld1_wait(tsum + (grp ^ 1u) * 32u));
+            const float inv_l = 1.0f / l_all;
+            uint32_t ov[2][32];
+            tmem_ld32(tO + grp * 64u + lane_off, ov[0]);
+            tmem_ld32(tO + grp * 64u + lane_off + 32u, ov[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(BAR(S_O_FREE));  // the next item's first P V may overwrite O
+            // O / l in bf16, 128-byte swizzled, into this group's box of the released V slot
+            const uint32_t stage = base + kSpV + bl * kTileBytes + grp * kBoxBytes;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t j = (uint32_t)(ch * 4 + q4);  // 16-byte chunk of this row's 128 bytes
+                    uint32_t w[4];
+#pragma unroll
+                    for (int k2 = 0; k2 < 4; ++k2)
+                        w[k2] = pack_bf16x2(__uint_as_float(ov[ch][q4 * 8 + 2 * k2]) * inv_l,
+                                            __uint_as_float(ov[ch][q4 * 8 + 2 * k2 + 1]) * inv_l);
+                    st_shared_v4(stage + (uint32_t)row * 128u + ((j ^ ((uint32_t)row & 7u)) << 4), w[0], w[1], w[2],
+                                 w[3]);
+                }
+            fence_proxy_async_smem();
+            mbar_arrive(BAR(S_STAGED0 + bl));  // the V producer stores the slot before it loads into it again
+            if (a.lse && grp == 0) a.lse[pd_grow] = (pd_m * c + lg2_approx(l_all)) * 0.6931471805599453f;
+            ++n_epi;
+            return true;
+        };
         SpItem it;
         for (int r = 0; ok && (ok = next_item(r, it, 1)) && !it.end; ++r) {
             if (it.count <= 0) continue;
@@ -469,60 +551,20 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(BAR(S_P_FULL0 + b));
+                // the previous item's epilogue, now that this item's first tile is out of the way
+                if (t == 0 && pend) {
+                    if (!(ok = epilogue())) break;
+                    pend = false;
+                }
             }
             if (!ok) break;
-            // Epilogue: full row sum from both groups, O / l for this group's 64 columns staged in the released V
-            // slot, one TMA store per group. The sums travel through the row-max buffer of the item's last tile:
-            // once the last P V is done, both groups have passed their reads of it (that P V needed both groups'
-            // P), and the next item's first tile uses the other buffer.
-            const uint32_t nl = n - 1;
-            if (!(ok = wait_bounded_warp(BAR(S_PV_DONE0 + (nl & 1u)), (nl >> 1) & 1u, lim))) break;
-            tc_fence_after();
-            float* const xsum = xmax + ((n_x - 1u) & 1u) * 256u;
-            xsum[grp * 128u + row] = l_run;
-            mbar_arrive(BAR(S_SUM_X));
-            if (!(ok = wait_bounded_warp(BAR(S_SUM_X), n_items & 1u, lim))) break;
-            const float l_all = l_run + xsum[(grp ^ 1u) * 128u + row];
-            const float inv_l = 1.0f / l_all;
-            uint32_t ov[2][32];
-            tmem_ld32(tO + grp * 64u + lane_off, ov[0]);
-            tmem_ld32(tO + grp * 64u + lane_off + 32u, ov[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(BAR(S_O_FREE));  // the next item's first P V may overwrite O
-            const uint32_t stage = base + kSpV + (nl & 1u) * kTileBytes + grp * kBoxBytes;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint32_t j = (uint32_t)(ch * 4 + q4);  // 16-byte chunk of this row's 128 bytes
-                    uint32_t w[4];
-#pragma unroll
-                    for (int k2 = 0; k2 < 4; ++k2)
-                        w[k2] = pack_bf16x2(__uint_as_float(ov[ch][q4 * 8 + 2 * k2]) * inv_l,
-                                            __uint_as_float(ov[ch][q4 * 8 + 2 * k2 + 1]) * inv_l);
-                    st_shared_v4(stage + (uint32_t)row * 128u + ((j ^ ((uint32_t)row & 7u)) << 4), w[0], w[1], w[2],
-                                 w[3]);
-                }
-            fence_proxy_async_smem();
-            mbar_arrive(BAR(S_ST_READY0 + grp));
-            if (!(ok = wait_bounded_warp(BAR(S_ST_READY0 + grp), n_items & 1u, lim))) break;
-            if (row == 0) {
-                tma_store_2d(&tmO, stage, 64 * (int)grp, it.h * a.Np + it.qb * kTcRows);
-                bulk_commit_group();
-                bulk_wait_read_all();
-                if (grp == 1) {
-                    mbar_arrive(BAR(S_ST_DONE));
-                } else if ((ok = wait_bounded(BAR(S_ST_DONE), n_items & 1u, lim))) {
-                    // both boxes have left the slot: hand it back to the V producer
-                    mbar_arrive(BAR(S_V_EMPTY0 + (nl & 1u)));
-                }
-            }
-            if (!(ok = __all_sync(0xffffffffu, ok))) break;
-            if (a.lse && grp == 0) a.lse[grow] = (m_raw * c + lg2_approx(l_all)) * 0.6931471805599453f;
-            ++n_items;
+            pend = true;
+            pd_grow = grow;
+            pd_m = m_raw;
+            pd_l = l_run;
+            pd_nl = n - 1;
         }
-        if (row == 0) bulk_wait_all();  // the O stores have landed before the CTA exits
+        if (ok && pend) epilogue();
     }
     // Teardown: every role has left its loop (normally or after a bounded wait ran out).
     tc_fence_before();
