@@ -6,12 +6,14 @@
 // blocks per 128 keys (1 for C = 128, 4 for C = 32).
 //
 // Shape of the work: one CTA per SM, one query block (item) at a time; keys are consumed in tiles of 256.
-//   S = Q K^T is one 128 x 256 tcgen05.mma tile (8 instructions of K = 16): N = 256 keeps the tensor core at its full
-//   rate, where N = 128 runs at about 60 %. TMEM holds S (columns 0..255), O (256..383) and P (384..511, bf16 pairs),
+//   S = Q K^T is one 128 x 256 tcgen05.mma tile (8 instructions of K = 16): N = 256 reads each Q fragment once for
+//   256 keys and needs half the instructions per key. TMEM holds S (columns 0..255), O (256..383) and P (384..511,
+//   bf16 pairs),
 //   so S is free as soon as the softmax has read it: the next QK^T overlaps this tile's softmax and P V.
 //   Two softmax warpgroups (warps 4..7 and 8..11) split the 256 columns; thread t of each owns query row t (TMEM lane
-//   t). They exchange their half-tile row maxima through shared memory, apply the same running max, keep their own
-//   partial row sums, rescale their own half of O, and write their own half of P. P V runs as two groups of eight
+//   t). Each also reads the other group's half of S, for the row max only: the max is exact, so both groups reach the
+//   same running max without an exchange. They keep their own partial row sums, rescale their own half of O, and
+//   write their own half of P. P V runs as two groups of eight
 //   N = 128 instructions (keys 0..127 and 128..255) with P read from TMEM and V from shared memory (MN-major).
 //   Warp 0 issues the TMA loads of Q (once per item) and K (single-buffered), warp 2 those of V (double-buffered),
 //   64 KB per 256-key tile; each box of a tile comes from its own lane. Warp 1 issues the MMAs and owns TMEM.
@@ -30,12 +32,12 @@ constexpr uint32_t kDnQ = 0;                       // Q tile, 32 KB
 constexpr uint32_t kDnK = 32768;                   // K tile of 256 keys, 64 KB: [d-half][256 rows][128 B]
 constexpr uint32_t kDnV = 98304;                   // V tiles, 2 x 64 KB, same layout; buffer 0 doubles as mass partials
 constexpr uint32_t kDnBar = 98304 + 2 * 65536;     // barriers, TMEM slot
-constexpr uint32_t kDnXchg = kDnBar + 256;         // [2 tile parity][2 groups][128] fp32 row maxima (row sums alias)
+constexpr uint32_t kDnXchg = kDnBar + 256;         // [2 item parity][2 groups][128] fp32 partial row sums
 constexpr uint32_t kDnSmem = kDnXchg + 2 * 2 * 128 * 4;  // 231680 bytes: needs a 1024-aligned dynamic base
 
 enum : uint32_t {
     D_Q_FULL = 0, D_Q_EMPTY, D_K_FULL, D_K_EMPTY, D_V_FULL0, D_V_FULL1, D_V_EMPTY0, D_V_EMPTY1, D_S_FULL, D_S_FREE,
-    D_P_FULL, D_PV_DONE, D_O_FREE, D_MAX_X, D_SUM_X, D_PART, D_PART2, D_MASS_DONE, D_MMA_DONE, D_COUNT
+    D_P_FULL, D_PV_DONE, D_O_FREE, D_SUM_X, D_PART, D_PART2, D_MASS_DONE, D_MMA_DONE, D_COUNT
 };
 
 template <bool WITH_MASS, int SUB>
@@ -52,14 +54,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t bar0 = base + kDnBar;
     auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kDnBar + D_COUNT * 8);
-    float* const xmax = reinterpret_cast<float*>(base_ptr + kDnXchg);           // [2 tile parity][2 group][128]
+    float* const xmax = reinterpret_cast<float*>(base_ptr + kDnXchg);           // [2 item parity][2 group][128]
     float* const part = reinterpret_cast<float*>(base_ptr + kDnV);              // [4 row groups][1024 blocks]
 
     const int warp = threadIdx.x >> 5;
     const uint32_t lane = lane_id();
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < D_COUNT; ++s) {
-            const bool wide = s == D_S_FREE || s == D_P_FULL || s == D_O_FREE || s == D_MAX_X || s == D_SUM_X ||
+            const bool wide = s == D_S_FREE || s == D_P_FULL || s == D_O_FREE || s == D_SUM_X ||
                               s == D_PART || s == D_PART2 || s == D_MASS_DONE;
             mbar_init(BAR(s), wide ? 256u : 1u);
         }
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t lane_off = (wl * 32u) << 16;
         const uint32_t tSg = tS + grp * 128u, tPg = tP + grp * 64u, tOg = tO + grp * 64u;
         const float c = a.scale_log2;
-        uint32_t n_s = 0, n_pv = 0, n_x = 0, n_items = 0, n_chunks = 0;
+        uint32_t n_s = 0, n_pv = 0, n_items = 0, n_chunks = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
             const int h = w / a.nq, qb = w - h * a.nq;
@@ -220,8 +222,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!(ok = wait_bounded_warp(BAR(D_S_FULL), n_s & 1u, lim))) break;
                 ++n_s;
                 tc_fence_after();
-                // One TMEM read of this group's 128 columns. S is released at once, so the next QK^T runs under
-                // this tile's softmax.
+                // The row max over the whole tile without a cross-group exchange: the other group's 128 columns are
+                // read first, 64 at a time, and only their maximum is kept (max is exact, so both groups agree).
+                float omax = -INFINITY;
+                {
+                    const int ovalid = a.N - (2 * t + (int)(1u - grp)) * 128;  // real keys in the other group's columns
+                    const uint32_t tSo = tS + (1u - grp) * 128u;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float o[64];
+                        tmem_ld32(tSo + lane_off + hh * 64u, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                        tmem_ld32(tSo + lane_off + hh * 64u + 32u, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                        tmem_wait_ld();
+                        if (ovalid < 128) {
+#pragma unroll
+                            for (int cc = 0; cc < 64; ++cc)
+                                if (hh * 64 + cc >= ovalid) o[cc] = -INFINITY;
+                        }
+                        float mx[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx[e] = fmax3(o[e], o[8 + e], o[16 + e]);
+#pragma unroll
+                        for (int cc = 24; cc < 64; cc += 16)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], o[cc + e], o[cc + 8 + e]);
+                        omax = fmaxf(omax, fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7]))));
+                    }
+                }
+                // This group's own 128 columns; S is released once both groups have read all of it, so the next QK^T
+                // runs under this tile's exponentials.
                 float s[128];
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch)
@@ -245,13 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], s[cc + e], s[cc + 8 + e]);
                     tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
                 }
-                // The row max over both groups' columns, exchanged through shared memory.
-                float* xm = xmax + (n_x & 1u) * 256u;
-                xm[grp * 128u + row] = tmax;
-                mbar_arrive(BAR(D_MAX_X));
-                if (!(ok = wait_bounded_warp(BAR(D_MAX_X), n_x & 1u, lim))) break;
-                ++n_x;
-                tmax = fmaxf(tmax, xm[(1u - grp) * 128u + row]);
+                tmax = fmaxf(tmax, omax);  // the tile max over all 256 columns
                 const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
                 const float alpha = (t > 0 && need) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
                 if (need) m_raw = tmax;
@@ -313,13 +336,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_arrive(BAR(D_P_FULL));
             }
             if (!ok) break;
-            // Epilogue: full row sum from both groups, O / l for this group's 64 columns, lse. The sums travel through
-            // the row-max buffer of the last tile: once the last P V is done, both groups have passed their reads of
-            // it (that P V needed both groups' P), and the next item's first tile uses the other buffer.
+            // Epilogue: full row sum from both groups, O / l for this group's 64 columns, lse. The sums go through a
+            // buffer per item parity: the item after next writes this one again only after the next item's P V,
+            // which needs both groups' P, so both have read these sums by then.
             if (!(ok = wait_bounded_warp(BAR(D_PV_DONE), n_pv & 1u, lim))) break;
             ++n_pv;
             tc_fence_after();
-            float* const xsum = xmax + ((n_x - 1u) & 1u) * 256u;
+            float* const xsum = xmax + (n_items & 1u) * 256u;
             xsum[grp * 128u + row] = l_run;
             mbar_arrive(BAR(D_SUM_X));
             if (!(ok = wait_bounded_warp(BAR(D_SUM_X), n_items & 1u, lim))) break;

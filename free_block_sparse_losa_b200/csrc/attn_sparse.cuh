@@ -19,9 +19,10 @@
 //            S_n = Q K^T (128 x 128, N = 128, Q read from TMEM) and O += P V of tile n - 1 (P from TMEM). With both
 //            A operands in TMEM, the MMAs read only K and V from shared memory.
 //   warps 4..11  softmax in two warpgroups that split each tile's keys (warps 4..7 keys 0..63, warps 8..11 keys
-//            64..127; thread t owns query row t = TMEM lane t). A group reads its half of S once and releases it, so
-//            the next QK^T runs under this tile's exponentials; the groups exchange their half-tile row maxima
-//            through shared memory, share one running max, keep their own partial sums and write their half of P.
+//            64..127; thread t owns query row t = TMEM lane t). A group reads the whole of S once (the other half
+//            only for its row max, which then needs no exchange: the max is exact, so both groups agree on it) and
+//            releases it, so the next QK^T runs under this tile's exponentials. The groups share one running max,
+//            keep their own partial sums and write their half of P.
 // TMEM: S columns 0..127, O 128..255, P_0 256..319, P_1 320..383 (bf16 pairs), Q_0 384..447, Q_1 448..511 (bf16
 // pairs, one buffer per item parity). O is rescaled in place only when a row's running max grows by more than 2^8
 // (the final division by the sum taken against the same reference keeps this exact); each group rescales its own 64
@@ -43,15 +44,14 @@ constexpr uint32_t kSpQ = 0;                              // 2 Q tiles
 constexpr uint32_t kSpK = 2 * kTileBytes;                 // 3 K tiles
 constexpr uint32_t kSpV = 5 * kTileBytes;                 // 2 V tiles (the second use: O staging)
 constexpr uint32_t kSpBar = 7 * kTileBytes;               // 48 barrier slots; the last holds the TMEM address
-constexpr uint32_t kSpX = kSpBar + 384;                   // [2 tile parity][2 groups][128] fp32 row maxima (sums alias)
-constexpr uint32_t kSpRing = kSpX + 2 * 2 * 128 * 4;      // 4 item records of 32 bytes
-constexpr uint32_t kSpSmem = kSpRing + 4 * 32;            // 231936 bytes: needs a 1024-aligned dynamic base
+constexpr uint32_t kSpRing = kSpBar + 384;                // 4 item records of 32 bytes
+constexpr uint32_t kSpSmem = kSpRing + 4 * 32;            // 229888 bytes: needs a 1024-aligned dynamic base
 constexpr int kSpKStages = 3;
 constexpr uint32_t kSpRingSlots = 4;
 
 enum : uint32_t {
     S_Q_FULL0 = 0, S_Q_EMPTY0 = 2, S_K_FULL0 = 4, S_K_EMPTY0 = 7, S_V_FULL0 = 10, S_V_EMPTY0 = 12, S_S_FULL = 14,
-    S_S_FREE = 16, S_P_FULL0 = 18, S_PV_DONE0 = 20, S_MAX_X = 22, S_SUM_X, S_O_FREE, S_STAGED0, S_IT_FULL0 = S_STAGED0 + 2,
+    S_S_FREE = 16, S_P_FULL0 = 18, S_PV_DONE0 = 20, S_SUM_R = 22, S_SUM_X, S_O_FREE, S_STAGED0, S_IT_FULL0 = S_STAGED0 + 2,
     S_IT_EMPTY0 = S_IT_FULL0 + kSpRingSlots, S_MMA_DONE = S_IT_EMPTY0 + kSpRingSlots, S_COUNT
 };
 constexpr int kSpThreads = 384;  // 12 warps: 0 Q/K TMA, 1 MMA, 2 V TMA, 3 work order, 4..11 softmax
@@ -126,7 +126,6 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     const uint32_t bar0 = base + kSpBar;
     auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sp_smem + kSpBar + 47 * 8);
-    float* const xmax = reinterpret_cast<float*>(sp_smem + kSpX);  // [2 tile parity][2 groups][128]
     SpItem* const ring = reinterpret_cast<SpItem*>(sp_smem + kSpRing);
 
     const int warp = threadIdx.x >> 5;
@@ -134,7 +133,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < S_COUNT; ++s) {
             uint32_t cnt = 1;
-            if (s == S_S_FREE || s == S_P_FULL0 || s == S_P_FULL0 + 1 || s == S_MAX_X || s == S_SUM_X ||
+            if (s == S_S_FREE || s == S_P_FULL0 || s == S_P_FULL0 + 1 || s == S_SUM_R || s == S_SUM_X ||
                 s == S_O_FREE || s == S_STAGED0 || s == S_STAGED0 + 1)
                 cnt = 256;
             else if (s >= S_IT_EMPTY0 && s < S_IT_EMPTY0 + kSpRingSlots)
@@ -397,11 +396,11 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         const int row = (int)(wl * 32u + lane);
         const uint32_t lane_off = (wl * 32u) << 16;
         const float c = a.scale_log2;
-        uint32_t n = 0, n_x = 0, n_epi = 0;
+        uint32_t n = 0, n_epi = 0;
         bool ok = true;
         // An item's epilogue waits until the next item's first tile is done: by then the item's last P V has
         // completed, where an immediate epilogue would sit waiting for it.
-        bool pend = false;
+        bool pend = false, sum_guard = false;  // sum_guard: the next P store waits for the last sum exchange's reads
         size_t pd_grow = 0;
         float pd_m = 0.0f, pd_l = 0.0f;
         uint32_t pd_nl = 0;
@@ -410,8 +409,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             if (!wait_bounded_warp(BAR(S_PV_DONE0 + bl), (pd_nl >> 1) & 1u, lim)) return false;
             tc_fence_after();
             // Full row sum: each group puts its partial sum into the first column of its half of the P buffer that
-            // the item's last P V has just released (rewritten only by tile pd_nl + 2, after both groups' next max
-            // exchange).
+            // the item's last P V has just released. Tile pd_nl + 2 rewrites that buffer; its P store waits on
+            // SUM_R, which both groups pass once they have read the other's sum.
             const uint32_t tsum = tP + bl * 64u + lane_off;
             tmem_st1(tsum + grp * 32u, __float_as_uint(pd_l));
             tmem_wait_st();
@@ -420,6 +419,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             if (!wait_bounded_warp(BAR(S_SUM_X), n_epi & 1u, lim)) return false;
             tc_fence_after();
             const float l_all = pd_l + __uint_as_float(tmem_ld1_wait(tsum + (grp ^ 1u) * 32u));
+            tc_fence_before();
+            mbar_arrive(BAR(S_SUM_R));
+            sum_guard = true;
             const float inv_l = 1.0f / l_all;
             uint32_t ov[2][32];
             tmem_ld32(tO + grp * 64u + lane_off, ov[0]);
@@ -462,6 +464,29 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 const uint32_t b = n & 1u;
                 if (!(ok = wait_bounded_warp(BAR(S_S_FULL), n & 1u, lim))) break;
                 tc_fence_after();
+                // The row max over the whole tile without a cross-group exchange: the other group's 64 columns are
+                // read first and only their maximum is kept (max is exact, so both groups get the same value).
+                float omax;
+                {
+                    const uint32_t oq0 = (kv4 >> (16 * (grp ^ 1u))) & 255u, oq1 = (kv4 >> (16 * (grp ^ 1u) + 8)) & 255u;
+                    float o[64];
+                    tmem_ld32(tS + (grp ^ 1u) * 64u + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                    tmem_ld32(tS + (grp ^ 1u) * 64u + lane_off + 32u, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                    tmem_wait_ld();
+                    if (oq0 != 32u || oq1 != 32u) {
+#pragma unroll
+                        for (int cc = 0; cc < 64; ++cc)
+                            if ((uint32_t)(cc & 31) >= (cc < 32 ? oq0 : oq1)) o[cc] = -INFINITY;
+                    }
+                    float mx[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx[e] = fmax3(o[e], o[8 + e], o[16 + e]);
+#pragma unroll
+                    for (int cc = 24; cc < 64; cc += 16)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], o[cc + e], o[cc + 8 + e]);
+                    omax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+                }
                 float s[64];
                 tmem_ld32(tS + grp * 64u + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
                 tmem_ld32(tS + grp * 64u + lane_off + 32u, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
@@ -484,13 +509,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                         for (int e = 0; e < 8; ++e) mx[e] = fmax3(mx[e], s[cc + e], s[cc + 8 + e]);
                     tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
                 }
-                // The tile's row max over both groups' columns, exchanged through shared memory.
-                float* const xm = xmax + (n_x & 1u) * 256u;
-                xm[grp * 128u + row] = tmax;
-                mbar_arrive(BAR(S_MAX_X));
-                if (!(ok = wait_bounded_warp(BAR(S_MAX_X), n_x & 1u, lim))) break;
-                ++n_x;
-                tmax = fmaxf(tmax, xm[(grp ^ 1u) * 128u + row]);
+                tmax = fmaxf(tmax, omax);  // the tile max over all 128 columns
                 // Reference max: raised only when the tile max exceeds it by more than 2^8 in the exp2 domain. A row
                 // that has seen no real key yet keeps a finite reference so that its weights are exact zeros.
                 const bool need = (t == 0) || (tmax - m_raw) * c > 8.0f;
@@ -546,7 +565,13 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                     }
                 }
                 // P buffer b was last read by P V of tile n - 2, issued before QK^T of tile n; this tile's S was
-                // written after it completed.
+                // written after it completed. After an epilogue it also holds the two groups' row sums until both
+                // have read them (this is then the first P store since, into that same buffer).
+                if (sum_guard) {
+                    if (!(ok = wait_bounded_warp(BAR(S_SUM_R), (n_epi - 1u) & 1u, lim))) break;
+                    tc_fence_after();
+                    sum_guard = false;
+                }
                 tmem_st32(tP + b * 64u + grp * 32u + lane_off, pw);
                 tmem_wait_st();
                 tc_fence_before();

@@ -17,7 +17,6 @@ constexpr uint32_t kBoxBytes = kTileBytes / 2;         // 16 KB: one 128-row x 6
 constexpr unsigned long long kDrainLimitNs = 2000000000ull;  // bound of the exit-path waits
 constexpr int kMaxMassBlocks = 1024;                   // key blocks per flush of the dense kernel's mass phase
 
-
 struct TcArgs {
     int H, N, Np, nq, nk, n_items;  // nk: 128-key tiles per head (Np / 128)
     int nkb;                        // key blocks of the selection (Np / C): nk for C = 128, 4 * nk for C = 32
@@ -76,33 +75,6 @@ __device__ __forceinline__ bool item_of_round(const TcArgs& a, int round, ItemIn
     return true;
 }
 
-// Block index of list entry e (clamped; the producer reports out-of-range entries).
-__device__ __forceinline__ int list_block(const TcArgs& a, const ItemInfo& it, int e) {
-    const int j = a.kv_idx[it.begin + e];
-    return (j < 0) ? 0 : (j >= a.nkb ? a.nkb - 1 : j);
-}
-
-// Real keys in each 32-key quarter of forward tile t, packed 8 bits per quarter. A quarter with no list entry (the
-// tail of a C = 32 list) has none; the ragged end of the sequence cuts the last block.
-template <int SUB>
-__device__ __forceinline__ uint32_t quarter_keys(const TcArgs& a, const ItemInfo& it, int t) {
-    uint32_t kv = 0;
-    if (SUB == 1 || !a.indptr) {
-        const int j128 = a.indptr ? list_block(a, it, t) : t;
-        const int kvalid = a.N - j128 * 128;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) kv |= (uint32_t)min(32, max(0, kvalid - 32 * g)) << (8 * g);
-    } else {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const int e = SUB * t + g;
-            if (e < it.count) kv |= (uint32_t)min(32, max(0, a.N - list_block(a, it, e) * 32)) << (8 * g);
-        }
-    }
-    return kv;
-}
-
-
 // 2^x on the FMA/ALU pipes, to take part of the load off the exp unit. Cody-Waite split x = n + f with n = round(x)
 // (the 1.5 * 2^23 shift leaves n in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial whose
 // coefficients minimise the maximum relative error on that interval (fitted by Lawson's iteratively reweighted least
@@ -111,18 +83,7 @@ __device__ __forceinline__ uint32_t quarter_keys(const TcArgs& a, const ItemInfo
 // use ex2_approx instead.
 constexpr float kExp2C0 = 0.9999992847442627f, kExp2C1 = 0.6931217908859253f, kExp2C2 = 0.240247443318367f,
                 kExp2C3 = 0.05591785907745361f, kExp2C4 = 0.009570102207362652f;
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(kExp2C4, f, kExp2C3);
-    p = fmaf(p, f, kExp2C2);
-    p = fmaf(p, f, kExp2C1);
-    p = fmaf(p, f, kExp2C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// exp2_poly on a pair of fp32 values with packed f32x2 arithmetic (the integer exponent update stays scalar).
+// The above on a pair of fp32 values with packed f32x2 arithmetic (the integer exponent update stays scalar).
 __device__ __forceinline__ void exp2_poly2(uint64_t xx, float& r0, float& r1) {
     float x0, x1;
     f2_unpack(xx, x0, x1);

@@ -130,7 +130,8 @@ losa_status launch_sparse_kernel(int grid, const CUtensorMap& tq, const CUtensor
     return launch_status();
 }
 
-// Tensor-core path: fills the argument block and launches one persistent CTA (two lanes) per SM.
+// Tensor-core path: fills the argument block and launches one persistent CTA per SM, the dense-step kernel
+// without a list, the sparse-step kernel with one.
 losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const void* k, const void* v, float scale,
                       const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
                       float* mass, cudaStream_t stream) {
