@@ -338,7 +338,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 #pragma unroll
                 for (uint32_t kk = 0; kk < 8; ++kk)
                     tc_mma_ts(tO, tP + b * 64u + kk * 8u, dV + kk * 128u, kIdPV, (pend_first && kk == 0) ? 0u : 1u);
-                // the last tile's V slot is released by the epilogue, after it has staged O there
+                // an item's last V slot comes back through the O staging: the V producer stores the item's O from it
+                // before refilling it
                 if (!pend_last) tc_commit(BAR(S_V_EMPTY0 + b));
                 tc_commit(BAR(S_PV_DONE0 + b));
                 pend = false;
