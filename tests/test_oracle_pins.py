@@ -34,6 +34,13 @@ def _rand_qkv(rng, H, N, Np, d, q_scale=1.0, k_scale=1.0):
     return q, k, v
 
 
+# Tolerance against the library's float64 attention. That reference (torch on the CPU) is not bitwise reproducible
+# from run to run under CPU load: 1 run in 160 measured here changed its log-sum-exp by up to 5.3e-10 (relative
+# 7e-11), while the oracle's output bits never changed. 1e-9 still sits many orders of magnitude below what a dropped
+# term, a wrong sign or a transposed operand produces (1e-3 and up); comparisons with closed forms stay at 1e-12.
+LIB_ATOL = 1e-9
+
+
 def _torch_attention(q, k, v, N, scale, key_mask=None):
     """Library routine: torch float64 SDPA over the first N keys (optionally a per-query key mask)."""
     qt = torch.from_numpy(q.astype(np.float64))
@@ -66,8 +73,8 @@ def test_dense_matches_library_sdpa():
     import oracle
     o, lse = oracle.dense(q, k, v, N, R, scale)
     ro, rl = _torch_attention(q[:, :N], k, v, N, scale)
-    np.testing.assert_allclose(_rows(o, R, Np // R, H, N), ro, rtol=0, atol=1e-12)
-    np.testing.assert_allclose(_rows(lse, R, Np // R, H, N), rl, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(_rows(o, R, Np // R, H, N), ro, rtol=0, atol=LIB_ATOL)
+    np.testing.assert_allclose(_rows(lse, R, Np // R, H, N), rl, rtol=0, atol=LIB_ATOL)
     # padded query rows carry no output
     assert np.isnan(o.reshape(H, Np, d)[:, N:]).all()
 
@@ -180,7 +187,7 @@ def test_mass_from_library_attention_probabilities():
             nr = rows.stop - rows.start
             for j in range(Np // C):
                 want = A[h, rows, j * C:min(N, (j + 1) * C)].sum() / nr
-                assert abs(m[h, i, j] - want) < 1e-12
+                assert abs(m[h, i, j] - want) < LIB_ATOL
 
 
 def test_mass_golden_worked_examples():
@@ -379,8 +386,8 @@ def test_sparse_matches_library_masked_sdpa():
     import oracle
     o, lse = oracle.sparse(q, k, v, N, R, C, 0.9, indptr, kv)
     ro, rl = _torch_attention(q[:, :N], k, v, N, 0.9, key_mask=mask[:, :N])
-    np.testing.assert_allclose(_rows(o, R, nq, H, N), ro, atol=1e-12)
-    np.testing.assert_allclose(_rows(lse, R, nq, H, N), rl, atol=1e-12)
+    np.testing.assert_allclose(_rows(o, R, nq, H, N), ro, atol=LIB_ATOL)
+    np.testing.assert_allclose(_rows(lse, R, nq, H, N), rl, atol=LIB_ATOL)
 
 
 def test_sparse_single_block_lists():
@@ -395,7 +402,7 @@ def test_sparse_single_block_lists():
         o, _ = oracle.sparse(q, k, v, N, R, R, 0.5, indptr, kv)
         sl = slice(j * R, (j + 1) * R)
         ro, _ = _torch_attention(q, k[:, sl], v[:, sl], R, 0.5)
-        np.testing.assert_allclose(o.reshape(1, Np, d), ro, atol=1e-12)
+        np.testing.assert_allclose(o.reshape(1, Np, d), ro, atol=LIB_ATOL)
 
 
 def test_sparse_tau_one_reproduces_dense():
