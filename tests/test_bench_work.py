@@ -1,0 +1,54 @@
+"""The benchmark's work model and roofline arithmetic, checked against invariants rather than restated formulas:
+with every block kept and no padding the sparse call does exactly the dense call's tensor work (at either key block
+size); the profile adds one more Q K^T pass over the same pairs; the selection moves the mass matrix plus its CSR
+output; a roofline fraction is achieved over peak. Runs without a GPU."""
+import dataclasses
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from losa_synth import CONFIGS  # noqa: E402
+
+
+@pytest.mark.parametrize("block_k", [0, 32])
+def test_full_lists_equal_dense_work(block_k):
+    cfg = dataclasses.replace(CONFIGS[1], block_k=block_k)
+    H, Np, d = cfg.heads, cfg.n_padded, cfg.head_dim
+    nnz = H * (Np // cfg.block) * (Np // cfg.kblock)  # every (item, key block)
+    w = bench.work_model(cfg, nnz)
+    # the dense-equivalent figure counts the N real tokens; with N = Np the two must agree exactly
+    assert w["sparse_flop"] == pytest.approx(w["dense_equiv_flop"] * (Np / cfg.n_tokens) ** 2, rel=1e-12)
+    assert w["sparse_flop"] == pytest.approx(4.0 * H * Np * Np * d, rel=1e-12)
+
+
+def test_profile_is_forward_plus_one_qk_pass():
+    cfg = CONFIGS[3]
+    w = bench.work_model(cfg, 0)
+    # forward: Q K^T and P V (2 flops per multiply-add each); masses: Q K^T once more
+    assert w["profile_flop"] == pytest.approx(w["dense_equiv_flop"] * 1.5, rel=1e-12)
+    assert w["profile_exp"] == pytest.approx(2.0 * cfg.heads * cfg.n_tokens ** 2, rel=1e-12)
+
+
+def test_select_bytes_are_mass_plus_csr():
+    cfg = CONFIGS[3]
+    rows = cfg.heads * cfg.n_blocks
+    for nnz in (0, 108056):
+        w = bench.work_model(cfg, nnz)
+        mass = 4 * rows * cfg.n_kblocks                 # fp32 mass matrix read once
+        csr = 4 * (nnz + rows + 1) + 4 * rows           # kv_block_idx, indptr, order
+        assert w["select_bytes"] == mass + csr
+
+
+def test_roofline_fraction_is_achieved_over_peak():
+    pk = {"bf16_tflops": 1618.0, "bf16_tflops_sustained": 1377.3, "hbm_gbs": 6551.4, "sm_max_mhz": 1965.0,
+          "source": "test"}
+    r = bench.roofline("k", "tensor", 2.0e12, 2.0e-3, pk, "TFLOP/s")  # 2e12 flop in 2 ms = 1000 TFLOP/s
+    assert r["achieved"] == pytest.approx(1000.0)
+    assert r["frac"] == pytest.approx(1000.0 / 1377.3, abs=1e-4)
+    r = bench.roofline("k", "hbm", 6.5514e9, 1.0e-3, pk, "GB/s")  # 6.55 GB in 1 ms = the measured peak
+    assert r["frac"] == pytest.approx(1.0, abs=1e-4)
