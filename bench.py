@@ -49,6 +49,16 @@ def peaks():
             "source": "fallback"}
 
 
+def bench_config(cfg, tau, world):
+    """The workload description both arms report (identical dicts for the same run)."""
+    elem = 2 if cfg.dtype == "bf16" else 4
+    qkv_mb = cfg.heads * cfg.n_padded * cfg.head_dim * elem / 1e6
+    return {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens, "n_padded": cfg.n_padded,
+            "head_dim": cfg.head_dim, "block": cfg.block, "block_k": cfg.kblock, "tau": tau,
+            "l2": "inputs larger than L2 (3 x %.0f MB of Q/K/V per layer)" % qkv_mb,
+            "parallelism": f"replicas x{world} (one independent layer per GPU)"}
+
+
 def work_model(cfg, nnz):
     """Algorithmic work per call. Tensor FLOPs count 2 per multiply-add; the dense-equivalent figure uses the
     real token count N, kept-block figures count whole 128 x 128 tiles."""
@@ -234,8 +244,7 @@ def run_reference(args, cfg):
     line = {"impl": "reference", "metric": METRIC, "value": c["value"], "unit": c["unit"], "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens,
-                       "head_dim": cfg.head_dim, "block": cfg.block, "tau": args.tau},
+            "config": bench_config(cfg, args.tau, args.gpus),
             "sparse_attn_ms": c["sparse_attn_ms_extrapolated"],
             "profile_select_ms": c["profile_select_ms_extrapolated"],
             "cpu_baseline": {"value": c["value"], "unit": c["unit"], "cores": c["cores"], "kind": "oracle",
@@ -425,10 +434,7 @@ def run_native(args, cfg):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
         "data": "synthetic (seeded grid-structured Q/K/V, see DESIGN.md)",
-        "config": {"workload": cfg.name, "heads": cfg.heads, "n_tokens": cfg.n_tokens, "n_padded": cfg.n_padded,
-                   "head_dim": cfg.head_dim, "block": cfg.block, "block_k": cfg.kblock, "tau": args.tau,
-                   "l2": "inputs larger than L2 (3 x %.0f MB of Q/K/V per layer)" % (q.numel() * 2 / 1e6),
-                   "parallelism": f"replicas x{world} (one independent layer per GPU)"},
+        "config": bench_config(cfg, args.tau, world),
         "sparse_attn_ms": round(per_sparse * 1e3, 3),
         "profile_ms": round(per_prof * 1e3, 3),
         "select_ms": round(per_sel * 1e3, 3),
