@@ -309,6 +309,40 @@ def test_select_brute_force_tiny():
             assert len(winners) == 1 and list(winners[0]) == kept
 
 
+def test_select_brute_force_nk_up_to_16():
+    """The same two facts for nk = 11..16, with the 2^nk subsets enumerated as bit masks."""
+    rng = np.random.default_rng(10)
+    import oracle
+    for trial, nk in enumerate((11, 12, 13, 14, 15, 16, 16, 16, 16)):
+        kind = trial % 3
+        if kind == 0:
+            m = rng.random(nk)
+        elif kind == 1:  # ties and zeros
+            m = rng.integers(0, 4, nk).astype(np.float64)
+            m[0] += 1
+        else:
+            m = rng.exponential(size=nk) ** 4
+        m = m / m.sum()
+        tau = float(rng.choice([0.5, 0.9, 0.99, 1.0]))
+        counts, idx = oracle.select(m[None], tau)
+        kept = [int(j) for j in idx[0, :counts[0]]]
+        u = _units(m).astype(np.int64)
+        T = int(math.ceil(tau * float(int(u.sum()))))
+        masks = np.arange(1 << nk, dtype=np.int64)
+        bits = (masks[:, None] >> np.arange(nk, dtype=np.int64)) & 1
+        sums = bits @ u
+        sizes = bits.sum(axis=1)
+        reach = sums >= T
+        best_size = int(sizes[reach].min())
+        best = reach & (sizes == best_size)
+        best_sum = int(sums[best].max())
+        assert counts[0] == best_size
+        assert int(u[kept].sum()) == best_sum
+        if len(set(m)) == nk:
+            winners = masks[best & (sums == best_sum)]
+            assert len(winners) == 1 and int(winners[0]) == sum(1 << j for j in kept)
+
+
 def test_select_topk_keeps_k_largest_with_index_ties():
     """Brute force: the kept set is the k largest masses, ties resolved toward lower indices; equal masses keep
     the first k indices; k >= nk keeps everything."""
