@@ -24,7 +24,9 @@
  *
  * Supported shapes: dtype BF16 with head_dim 128, block_q = 128 and block_k = 128 or 32 (tensor-core path; 32 is the
  * LoSA page's key-block size), or dtype F32 with head_dim 64 or 128 and block_q = block_k in {32, 64, 128} (exact fp32
- * path for small checks).
+ * path for small checks). Size limits: the tensor-core path takes Np <= 131072 (1024 blocks of 128 tokens per head);
+ * the selection calls take nk <= 8192 key blocks per row and H * nq <= 32768 items per call. Any other valid shape
+ * returns LOSA_ERR_UNSUPPORTED before anything is launched.
  */
 #ifndef LOSA_H
 #define LOSA_H

@@ -89,9 +89,19 @@ def test_capacity_and_unsupported(lib):
                          raise_on_error=False) == -3
     assert L.losa_select(s, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=rows * nk, ws_bytes=ws - 1, stream=0,
                          raise_on_error=False) == -3
-    # bf16 is implemented for head_dim 128 with 128-blocks only
-    s64 = L.make_shape(2, 1000, 1024, 64, 128, 128, "bf16")
-    assert L.losa_dense_profile(s64, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, None, stream=0, raise_on_error=False) == -2
+    # bf16 is implemented for head_dim 128, block_q 128 and block_k 128 or 32, up to 1024 blocks of 128 per head
+    for s_bad in (L.make_shape(2, 1000, 1024, 64, 128, 128, "bf16"),
+                  L.make_shape(2, 1000, 1024, 128, 128, 64, "bf16"),
+                  L.make_shape(2, 1000, 1024, 128, 64, 64, "bf16"),
+                  L.make_shape(1, 131100, 131200, 128, 128, 128, "bf16")):
+        assert L.losa_dense_profile(s_bad, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, None, stream=0,
+                                    raise_on_error=False) == -2
+        assert L.losa_sparse_attn(s_bad, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, None, FAKE, stream=0,
+                                  raise_on_error=False) == -2
+    # more than 8192 key blocks per selection row
+    wide = L.make_shape(1, 262200, 262272, 128, 128, 32, "bf16")
+    assert L.losa_select(wide, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40,
+                         ws_bytes=L.losa_select_workspace_bytes(wide), stream=0, raise_on_error=False) == -2
     # more items than one selection call orders
     big = L.make_shape(300, 130000, 130048, 128, 128, 128, "bf16")
     wsb = L.losa_select_workspace_bytes(big)
