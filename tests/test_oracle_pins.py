@@ -360,6 +360,22 @@ def test_select_topk_keeps_k_largest_with_index_ties():
     assert list(idx[0, :counts[0]]) == [0, 1, 2]
 
 
+def test_select_tiny_tau_keeps_the_heaviest_block():
+    """Any tau > 0 keeps at least one block, and a tau below the largest mass keeps exactly the heaviest block
+    (the lowest index among equal maxima); a row of all-equal masses keeps block 0."""
+    rng = np.random.default_rng(12)
+    import oracle
+    m = rng.exponential(size=(40, 25)) ** 3
+    m[5] = 1.0
+    m[6, 3] = m[6, 17] = m[6].max() * 2.0
+    m /= m.sum(axis=1, keepdims=True)
+    for tau in (1e-300, 1e-12, 1e-3):
+        counts, idx = oracle.select(m, tau)
+        assert (counts == 1).all()
+        assert idx[:, 0].tolist() == np.argmax(m, axis=1).tolist()
+    assert idx[5, 0] == 0 and idx[6, 0] == 3
+
+
 def test_select_rejects_bad_tau():
     import oracle
     m = np.full((1, 4), 0.25)
