@@ -32,7 +32,6 @@ if ROOT not in sys.path:
 
 from losa_synth import CONFIGS, make_layer, sample_items  # noqa: E402
 
-WORKLOADS = {"hunyuan720": 3, "wan14b720": 2, "wan1.3b480": 1, "tiny": 0, "loop": 4}
 METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select ms"
 KERNELS_PER_STEP = {"dense_profile": 1, "select": 3, "sparse_attn": 1}
 
@@ -433,7 +432,7 @@ def run_native(args, cfg):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s (dense-equivalent, sparse attention)",
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-        "data": "synthetic (seeded grid-structured Q/K/V, see DESIGN.md)",
+        "data": "synthetic: seeded grid-structured Q/K/V (per-head random Fourier locality, sink keys, padded tail)",
         "config": bench_config(cfg, args.tau, world),
         "sparse_attn_ms": round(per_sparse * 1e3, 3),
         "profile_ms": round(per_prof * 1e3, 3),
@@ -598,7 +597,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="hunyuan720")
+    ap.add_argument("--workload", choices=sorted(CONFIGS), default="hunyuan720")
     ap.add_argument("--tau", type=float, default=0.99)
     ap.add_argument("--block-k", type=int, default=0, choices=[0, 32, 128],
                     help="key block size C (0: the workload's, 128; 32 is the LoSA page's setup)")
@@ -611,7 +610,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    cfg = CONFIGS[WORKLOADS[args.workload]]
+    cfg = CONFIGS[args.workload]
     if args.block_k:
         import dataclasses
         cfg = dataclasses.replace(cfg, block_k=args.block_k)

@@ -77,16 +77,16 @@ class LayerConfig:
 
 
 CONFIGS = {
-    0: LayerConfig("tiny-4x8x8-h2-d64-f32", heads=2, grid=(4, 8, 8), head_dim=64, block=64, dtype="f32",
+    "tiny": LayerConfig("tiny-4x8x8-h2-d64-f32", heads=2, grid=(4, 8, 8), head_dim=64, block=64, dtype="f32",
                    amplitude=3.0, ell_fixed=(2.0, 3.0, 3.0), n_sinks=0, seed=0, taus=(0.9, 0.99, 1.0)),
-    1: LayerConfig("wan2.1-1.3b-480p-21x30x52-h12", heads=12, grid=(21, 30, 52), head_dim=128, block=128,
+    "wan1.3b480": LayerConfig("wan2.1-1.3b-480p-21x30x52-h12", heads=12, grid=(21, 30, 52), head_dim=128, block=128,
                    dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=2, seed=1,
                    taus=(0.9, 0.95, 0.99, 1.0)),
-    2: LayerConfig("wan2.1-14b-720p-21x45x80-h40", heads=40, grid=(21, 45, 80), head_dim=128, block=128,
+    "wan14b720": LayerConfig("wan2.1-14b-720p-21x45x80-h40", heads=40, grid=(21, 45, 80), head_dim=128, block=128,
                    dtype="bf16", amplitude=4.0, ell_range=(1.0, 12.0), n_sinks=2, seed=2, taus=(0.99,)),
-    3: LayerConfig("hunyuanvideo-720p-33x45x80-h24", heads=24, grid=(33, 45, 80), head_dim=128, block=128,
+    "hunyuan720": LayerConfig("hunyuanvideo-720p-33x45x80-h24", heads=24, grid=(33, 45, 80), head_dim=128, block=128,
                    dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=2, seed=3, taus=(0.99,)),
-    4: LayerConfig("wan2.1-1.3b-480p-loop-30layers-h12", heads=12, grid=(21, 30, 52), head_dim=128, block=128,
+    "loop": LayerConfig("wan2.1-1.3b-480p-loop-30layers-h12", heads=12, grid=(21, 30, 52), head_dim=128, block=128,
                    dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=2, seed=4, layers=30,
                    taus=(0.99,), extra={"steps": 50, "drift": 0.02}),
 }
@@ -166,9 +166,10 @@ def _gen_head(cfg: LayerConfig, ss: np.random.SeedSequence, pos: np.ndarray):
     return out, float(ell[0]) if cfg.ell_fixed is None else ell.copy(), sinks
 
 
-def make_layer(cfg: LayerConfig | int, layer: int = 0, threads: int = 8) -> Layer:
-    """Generate layer `layer` of a config (layer > 0 only for multi-layer configs)."""
-    if isinstance(cfg, int):
+def make_layer(cfg: LayerConfig | str, layer: int = 0, threads: int = 8) -> Layer:
+    """Generate layer `layer` of a config, given as a LayerConfig or a workload name (layer > 0 only for
+    multi-layer configs)."""
+    if isinstance(cfg, str):
         cfg = CONFIGS[cfg]
     if not 0 <= layer < cfg.layers:
         raise ValueError("layer out of range")

@@ -17,7 +17,7 @@ from losa_synth import CONFIGS  # noqa: E402
 
 @pytest.mark.parametrize("block_k", [0, 32])
 def test_full_lists_equal_dense_work(block_k):
-    cfg = dataclasses.replace(CONFIGS[1], block_k=block_k)
+    cfg = dataclasses.replace(CONFIGS["wan1.3b480"], block_k=block_k)
     H, Np, d = cfg.heads, cfg.n_padded, cfg.head_dim
     nnz = H * (Np // cfg.block) * (Np // cfg.kblock)  # every (item, key block)
     w = bench.work_model(cfg, nnz)
@@ -27,7 +27,7 @@ def test_full_lists_equal_dense_work(block_k):
 
 
 def test_profile_is_forward_plus_one_qk_pass():
-    cfg = CONFIGS[3]
+    cfg = CONFIGS["hunyuan720"]
     w = bench.work_model(cfg, 0)
     # forward: Q K^T and P V (2 flops per multiply-add each); masses: Q K^T once more
     assert w["profile_flop"] == pytest.approx(w["dense_equiv_flop"] * 1.5, rel=1e-12)
@@ -35,7 +35,7 @@ def test_profile_is_forward_plus_one_qk_pass():
 
 
 def test_select_bytes_are_mass_plus_csr():
-    cfg = CONFIGS[3]
+    cfg = CONFIGS["hunyuan720"]
     rows = cfg.heads * cfg.n_blocks
     for nnz in (0, 108056):
         w = bench.work_model(cfg, nnz)

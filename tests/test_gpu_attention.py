@@ -36,7 +36,7 @@ SMALL = {
     "bf16-1x(1x1x77)-one-block": LayerConfig("one-block", heads=1, grid=(1, 1, 77), head_dim=128, block=128,
                                              dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=1,
                                              seed=102, taus=(0.99,)),
-    "f32-tiny": CONFIGS[0],
+    "f32-tiny": CONFIGS["tiny"],
     # the LoSA page's block shape: 128-row query blocks, 32-key blocks
     "bf16-C32-2x(4x16x16)": LayerConfig("small-bf16-c32", heads=2, grid=(4, 16, 16), head_dim=128, block=128,
                                         block_k=32, dtype="bf16", amplitude=4.0, ell_range=(1.0, 8.0), n_sinks=2,
@@ -100,14 +100,15 @@ def test_small_full_comparison(name, oracle_mod):
     _pipeline(SMALL[name], None, oracle_mod)
 
 
-@pytest.mark.parametrize("cfg_id,block_k", [(1, 128), (2, 128), (3, 128), (1, 32), (3, 32)])
-def test_full_size_sampled(cfg_id, block_k, oracle_mod):
+@pytest.mark.parametrize("workload,block_k", [("wan1.3b480", 128), ("wan14b720", 128), ("hunyuan720", 128),
+                                              ("wan1.3b480", 32), ("hunyuan720", 32)])
+def test_full_size_sampled(workload, block_k, oracle_mod):
     import dataclasses
-    cfg = dataclasses.replace(CONFIGS[cfg_id], block_k=block_k)
+    cfg = dataclasses.replace(CONFIGS[workload], block_k=block_k)
     layer = make_layer(cfg)
     # 64 seeded items, including the tail block of head 0 and the query blocks holding head 0's sink tokens
     sink_items = [int(t) // cfg.block for t in layer.sinks[0]]
-    items = sample_items(cfg, 64, seed=cfg_id, must_include=sink_items)
+    items = sample_items(cfg, 64, seed=cfg.seed, must_include=sink_items)
     _pipeline(cfg, items, oracle_mod, layer=layer)
 
 

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 def test_frozen_pattern_reused_on_drifted_inputs(oracle_mod):
     require_gpu()
-    cfg = CONFIGS[4]  # Wan2.1-480p-shaped layers; 2 of its 30 layers, 4 steps
+    cfg = CONFIGS["loop"]  # Wan2.1-480p-shaped layers; 2 of its 30 layers, 4 steps
     layers = [make_layer(cfg, li) for li in range(2)]
     drift = Drift(cfg, layers, seed=cfg.seed)
     scale = 1.0 / math.sqrt(cfg.head_dim)

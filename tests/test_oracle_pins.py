@@ -473,7 +473,7 @@ def test_sparse_tau_one_reproduces_dense():
 
 def test_recall_at_construction_reaches_tau():
     """Selection on exact masses retains at least theta of every row's mass (by construction)."""
-    layer = make_layer(0)
+    layer = make_layer("tiny")
     cfg = layer.cfg
     import oracle
     q, k = layer.all_f32("q"), layer.all_f32("k")
@@ -499,12 +499,12 @@ def test_bf16_rounding_matches_torch():
 
 
 def test_generator_is_seeded_and_padded():
-    a, b = make_layer(0), make_layer(0)
+    a, b = make_layer("tiny"), make_layer("tiny")
     np.testing.assert_array_equal(a.q, b.q)
     np.testing.assert_array_equal(a.k, b.k)
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     assert a.q.shape == (cfg.heads, cfg.n_padded, cfg.head_dim)
     # config 1 geometry: 21*30*52 = 32760 tokens, padded to 32768 with zero rows
-    c1 = CONFIGS[1]
+    c1 = CONFIGS["wan1.3b480"]
     assert (c1.n_tokens, c1.n_padded, c1.n_blocks) == (32760, 32768, 256)
-    assert CONFIGS[3].n_padded == 118912 and CONFIGS[2].n_padded == 75648
+    assert CONFIGS["hunyuan720"].n_padded == 118912 and CONFIGS["wan14b720"].n_padded == 75648
