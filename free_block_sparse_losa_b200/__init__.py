@@ -81,16 +81,41 @@ def load():
     return L
 
 
-def _ptr(t):
-    if t is None:
-        return None
-    if isinstance(t, int):
-        return t
-    if not t.is_cuda:
-        raise ValueError("expected a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError("expected a contiguous tensor")
-    return t.data_ptr()
+def _dims(shape):
+    """(H, Np, d, nq, nk) of a shape; 0 for a block count whose block size is not positive."""
+    nq = shape.n_padded // shape.block_q if shape.block_q > 0 else 0
+    nk = shape.n_padded // shape.block_k if shape.block_k > 0 else 0
+    return max(shape.heads, 0), max(shape.n_padded, 0), max(shape.head_dim, 0), max(nq, 0), max(nk, 0)
+
+
+def _token_dtype(shape):
+    return {DTYPE_F32: "float32", DTYPE_BF16: "bfloat16"}.get(shape.dtype)
+
+
+def _ptrs(*specs):
+    """Device pointers of arguments given as (value, name, dtype, numel). None stays NULL and an int is taken as a raw
+    device pointer (the caller vouches for its size). A tensor must have the expected dtype (if given), hold at least
+    `numel` elements (if given), be contiguous and live on the current CUDA device, so that a wrong buffer is refused
+    here instead of being read or written out of bounds. The dtype, size and layout of every argument are checked
+    before any argument's device."""
+    tensors = [(t, name) for t, name, _, _ in specs if t is not None and not isinstance(t, int)]
+    if tensors:
+        import torch
+    for t, name, dtype, numel in specs:
+        if t is None or isinstance(t, int):
+            continue
+        if dtype is not None and t.dtype != getattr(torch, dtype):
+            raise ValueError(f"{name}: expected torch.{dtype}, got {t.dtype}")
+        if numel is not None and t.numel() < numel:
+            raise ValueError(f"{name}: holds {t.numel()} elements, the shape needs {numel}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous tensor")
+    for t, name in tensors:
+        if not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA tensor")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name}: lives on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
+    return tuple(t if (t is None or isinstance(t, int)) else t.data_ptr() for t, _, _, _ in specs)
 
 
 def _stream(stream):
@@ -109,8 +134,12 @@ def _check(status: int, where: str, raise_on_error: bool):
 
 
 def losa_dense_profile(shape, q, k, v, scale, o, lse=None, mass=None, stream=None, raise_on_error=True):
-    st = load().losa_dense_profile(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(o), _ptr(lse),
-                                   _ptr(mass), _stream(stream))
+    H, Np, d, nq, nk = _dims(shape)
+    tdt = _token_dtype(shape)
+    pq, pk, pv, po, pl, pm = _ptrs((q, "q", tdt, H * Np * d), (k, "k", tdt, H * Np * d), (v, "v", tdt, H * Np * d),
+                                   (o, "o", tdt, H * Np * d), (lse, "lse", "float32", H * Np),
+                                   (mass, "mass", "float32", H * nq * nk))
+    st = load().losa_dense_profile(ctypes.byref(shape), pq, pk, pv, float(scale), po, pl, pm, _stream(stream))
     return _check(st, "losa_dense_profile", raise_on_error)
 
 
@@ -118,37 +147,66 @@ def losa_select_workspace_bytes(shape) -> int:
     return int(load().losa_select_workspace_bytes(ctypes.byref(shape)))
 
 
+def _select_args(shape, mass, indptr, kv_block_idx, order, idx_capacity, workspace=None, ws_bytes=None):
+    """Pointers of the selection calls' arguments, the index capacity and the workspace size."""
+    H, _, _, nq, nk = _dims(shape)
+    if idx_capacity is None:
+        if isinstance(kv_block_idx, int):
+            raise ValueError("kv_block_idx: a raw pointer needs idx_capacity")
+        cap, idx_numel = kv_block_idx.numel(), None
+    else:
+        cap = idx_numel = int(idx_capacity)
+    wsb = None
+    if workspace is not None:
+        if isinstance(workspace, int):
+            if ws_bytes is None:
+                raise ValueError("workspace: a raw pointer needs ws_bytes")
+            wsb = int(ws_bytes)
+        else:
+            have = workspace.numel() * workspace.element_size()
+            wsb = have if ws_bytes is None else int(ws_bytes)
+            if have < wsb:
+                raise ValueError(f"workspace: holds {have} bytes, ws_bytes says {wsb}")
+    ptrs = _ptrs((mass, "mass", "float32", H * nq * nk), (indptr, "indptr", "int32", H * nq + 1),
+                 (kv_block_idx, "kv_block_idx", "int32", idx_numel), (order, "order", "int32", H * nq),
+                 (workspace, "workspace", None, None))
+    return ptrs, cap, wsb
+
+
 def losa_select(shape, mass, tau, indptr, kv_block_idx, order, workspace, idx_capacity=None, ws_bytes=None,
                 stream=None, raise_on_error=True):
-    cap = kv_block_idx.numel() if idx_capacity is None else idx_capacity
-    wsb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
-    st = load().losa_select(ctypes.byref(shape), _ptr(mass), float(tau), _ptr(indptr), _ptr(kv_block_idx), int(cap),
-                            _ptr(order), _ptr(workspace), int(wsb), _stream(stream))
+    (pm, pi, pk, po, pw), cap, wsb = _select_args(shape, mass, indptr, kv_block_idx, order, idx_capacity, workspace,
+                                                  ws_bytes)
+    st = load().losa_select(ctypes.byref(shape), pm, float(tau), pi, pk, cap, po, pw, wsb, _stream(stream))
     return _check(st, "losa_select", raise_on_error)
 
 
 def losa_select_topk(shape, mass, k_blocks, indptr, kv_block_idx, order, workspace, idx_capacity=None, ws_bytes=None,
                      stream=None, raise_on_error=True):
-    cap = kv_block_idx.numel() if idx_capacity is None else idx_capacity
-    wsb = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
-    st = load().losa_select_topk(ctypes.byref(shape), _ptr(mass), int(k_blocks), _ptr(indptr), _ptr(kv_block_idx),
-                                 int(cap), _ptr(order), _ptr(workspace), int(wsb), _stream(stream))
+    (pm, pi, pk, po, pw), cap, wsb = _select_args(shape, mass, indptr, kv_block_idx, order, idx_capacity, workspace,
+                                                  ws_bytes)
+    st = load().losa_select_topk(ctypes.byref(shape), pm, int(k_blocks), pi, pk, cap, po, pw, wsb, _stream(stream))
     return _check(st, "losa_select_topk", raise_on_error)
 
 
 def losa_select_noalloc(shape, mass, tau, indptr, kv_block_idx, order, idx_capacity=None, stream=None,
                         raise_on_error=True):
     """losa_select with the library's fixed device scratch instead of a caller workspace (see include/losa.h)."""
-    cap = kv_block_idx.numel() if idx_capacity is None else idx_capacity
-    st = load().losa_select_noalloc(ctypes.byref(shape), _ptr(mass), float(tau), _ptr(indptr), _ptr(kv_block_idx),
-                                    int(cap), _ptr(order), _stream(stream))
+    (pm, pi, pk, po, _), cap, _ = _select_args(shape, mass, indptr, kv_block_idx, order, idx_capacity)
+    st = load().losa_select_noalloc(ctypes.byref(shape), pm, float(tau), pi, pk, cap, po, _stream(stream))
     return _check(st, "losa_select_noalloc", raise_on_error)
 
 
 def losa_sparse_attn(shape, q, k, v, scale, indptr, kv_block_idx, order, o, lse=None, stream=None,
                      raise_on_error=True):
-    st = load().losa_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(indptr),
-                                 _ptr(kv_block_idx), _ptr(order), _ptr(o), _ptr(lse), _stream(stream))
+    H, Np, d, nq, _ = _dims(shape)
+    tdt = _token_dtype(shape)
+    pq, pk, pv, pi, px, po, pout, pl = _ptrs(
+        (q, "q", tdt, H * Np * d), (k, "k", tdt, H * Np * d), (v, "v", tdt, H * Np * d),
+        (indptr, "indptr", "int32", H * nq + 1), (kv_block_idx, "kv_block_idx", "int32", None),
+        (order, "order", "int32", H * nq), (o, "o", tdt, H * Np * d), (lse, "lse", "float32", H * Np))
+    st = load().losa_sparse_attn(ctypes.byref(shape), pq, pk, pv, float(scale), pi, px, po, pout, pl,
+                                 _stream(stream))
     return _check(st, "losa_sparse_attn", raise_on_error)
 
 

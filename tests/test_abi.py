@@ -114,3 +114,42 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(RuntimeError):
         L.load()
+
+
+def test_binding_refuses_wrong_tensors_before_the_call(lib):
+    """The binding checks each tensor against the shape (dtype, element count, layout, device) and raises before
+    anything reaches the library, so a wrong buffer is never read or written out of bounds."""
+    import torch
+    H, N, Np, d, R = 2, 1000, 1024, 128, 128
+    s = L.make_shape(H, N, Np, d, R, R, "bf16")
+    tok = lambda n=H * Np * d, dt=torch.bfloat16: torch.empty(n, dtype=dt)  # noqa: E731
+    i32 = lambda n: torch.empty(n, dtype=torch.int32)  # noqa: E731
+    f32 = lambda n: torch.empty(n, dtype=torch.float32)  # noqa: E731
+    rows, nk = H * (Np // R), Np // R
+    with pytest.raises(ValueError, match="q: expected torch.bfloat16"):
+        L.losa_dense_profile(s, tok(dt=torch.float16), tok(), tok(), 0.1, tok(), f32(H * Np), None)
+    with pytest.raises(ValueError, match="v: holds"):
+        L.losa_dense_profile(s, tok(), tok(), tok(H * Np * d - 1), 0.1, tok(), f32(H * Np), None)
+    with pytest.raises(ValueError, match="mass: holds"):
+        L.losa_dense_profile(s, tok(), tok(), tok(), 0.1, tok(), f32(H * Np), f32(rows * nk - 1))
+    with pytest.raises(ValueError, match="o: expected a contiguous"):
+        L.losa_dense_profile(s, tok(), tok(), tok(), 0.1, tok(2 * H * Np * d)[::2], f32(H * Np), None)
+    with pytest.raises(ValueError, match="q: expected a CUDA tensor"):
+        L.losa_dense_profile(s, tok(), tok(), tok(), 0.1, tok(), f32(H * Np), None)
+    with pytest.raises(ValueError, match="indptr: expected torch.int32"):
+        L.losa_select(s, f32(rows * nk), 0.99, torch.empty(rows + 1, dtype=torch.int64), i32(rows * nk), i32(rows),
+                      torch.empty(64, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="order: holds"):
+        L.losa_select(s, f32(rows * nk), 0.99, i32(rows + 1), i32(rows * nk), i32(rows - 1),
+                      torch.empty(64, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="kv_block_idx: holds"):
+        L.losa_select(s, f32(rows * nk), 0.99, i32(rows + 1), i32(rows * nk), i32(rows),
+                      torch.empty(64, dtype=torch.uint8), idx_capacity=rows * nk + 1)
+    with pytest.raises(ValueError, match="workspace: holds"):
+        L.losa_select(s, f32(rows * nk), 0.99, i32(rows + 1), i32(rows * nk), i32(rows),
+                      torch.empty(64, dtype=torch.uint8), ws_bytes=65)
+    with pytest.raises(ValueError, match="a raw pointer needs idx_capacity"):
+        L.losa_select_noalloc(s, FAKE, 0.99, FAKE, FAKE, FAKE)
+    with pytest.raises(ValueError, match="lse: expected torch.float32"):
+        L.losa_sparse_attn(s, tok(), tok(), tok(), 0.1, i32(rows + 1), i32(1), None, tok(),
+                           torch.empty(H * Np, dtype=torch.float64))
