@@ -17,35 +17,42 @@ _LIB = os.path.join(_HERE, "liblosa_oracle.so")
 _lib = None
 
 
+def compile_command(src: str, out: str) -> list:
+    return ["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared", "-o", out, src]
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle with the system C++ compiler (portable flags: it may run on another host)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared", "-o", _LIB + ".tmp", _SRC]
-        subprocess.run(cmd, check=True)
+        subprocess.run(compile_command(_SRC, _LIB + ".tmp"), check=True)
         os.replace(_LIB + ".tmp", _LIB)
     return _LIB
+
+
+def bind(path: str):
+    """Load a compiled oracle library and declare its entry points."""
+    L = ctypes.CDLL(path)
+    i32, f64, vp = ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+    L.oracle_num_threads.restype = i32
+    L.oracle_dense.argtypes = [i32, i32, i32, i32, i32, f64, vp, vp, vp, i32, vp, vp, vp]
+    L.oracle_mass.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, i32, vp, vp]
+    L.oracle_select_f32.argtypes = [i32, i32, vp, f64, vp, vp]
+    L.oracle_select_f64.argtypes = [i32, i32, vp, f64, vp, vp]
+    L.oracle_select_topk.argtypes = [i32, i32, vp, i32, vp, vp]
+    L.oracle_lpt_order.argtypes = [i32, vp, vp]
+    L.oracle_sparse.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, vp, vp, vp, i32, vp, vp, vp]
+    L.oracle_recall.argtypes = [i32, i32, vp, vp, vp, vp]
+    L.oracle_recall.restype = f64
+    for name in ("oracle_dense", "oracle_mass", "oracle_select_f32", "oracle_select_f64", "oracle_select_topk",
+                 "oracle_lpt_order", "oracle_sparse"):
+        getattr(L, name).restype = i32
+    return L
 
 
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
-        i32, f64, vp = ctypes.c_int, ctypes.c_double, ctypes.c_void_p
-        L.oracle_num_threads.restype = i32
-        L.oracle_dense.argtypes = [i32, i32, i32, i32, i32, f64, vp, vp, vp, i32, vp, vp, vp]
-        L.oracle_mass.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, i32, vp, vp]
-        L.oracle_select_f32.argtypes = [i32, i32, vp, f64, vp, vp]
-        L.oracle_select_f64.argtypes = [i32, i32, vp, f64, vp, vp]
-        L.oracle_select_topk.argtypes = [i32, i32, vp, i32, vp, vp]
-        L.oracle_lpt_order.argtypes = [i32, vp, vp]
-        L.oracle_sparse.argtypes = [i32, i32, i32, i32, i32, i32, f64, vp, vp, vp, vp, vp, i32, vp, vp, vp]
-        L.oracle_recall.argtypes = [i32, i32, vp, vp, vp, vp]
-        L.oracle_recall.restype = f64
-        for name in ("oracle_dense", "oracle_mass", "oracle_select_f32", "oracle_select_f64", "oracle_select_topk",
-                     "oracle_lpt_order", "oracle_sparse"):
-            getattr(L, name).restype = i32
-        _lib = L
+        _lib = bind(build())
     return _lib
 
 

@@ -487,6 +487,27 @@ def test_recall_at_construction_reaches_tau():
         assert oracle.recall(m, indptr, kv) >= tau - 1e-12
 
 
+def test_recall_closed_forms():
+    """Recall (Motivation Summary: retained mass over total mass of the rows) of patterns whose value is known:
+    every block gives 1, block j alone gives column j's share, and a subset of rows counts only those rows."""
+    rng = np.random.default_rng(16)
+    import oracle
+    m = rng.random((6, 5))
+    full = np.tile(np.arange(5, dtype=np.int32), 6)
+    assert abs(oracle.recall(m, np.arange(0, 31, 5, dtype=np.int32), full) - 1.0) < 1e-15
+    for j in range(5):
+        one = np.full(6, j, np.int32)
+        assert abs(oracle.recall(m, np.arange(7, dtype=np.int32), one) - m[:, j].sum() / m.sum()) < 1e-14
+    # rows 4 and 1 of a pattern where row r keeps blocks 0..r-1 (row 0 keeps block 0)
+    lists = [np.arange(max(r, 1), dtype=np.int32) for r in range(6)]
+    indptr = np.zeros(7, np.int32)
+    indptr[1:] = np.cumsum([len(x) for x in lists])
+    kv = np.concatenate(lists)
+    sub = m[[4, 1]]
+    want = (sub[0, :4].sum() + sub[1, :1].sum()) / sub.sum()
+    assert abs(oracle.recall(sub, indptr, kv, rows=[4, 1]) - want) < 1e-14
+
+
 # ------------------------------------------------------------------------------------------- generator
 
 def test_bf16_rounding_matches_torch():
