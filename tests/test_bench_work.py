@@ -52,3 +52,24 @@ def test_roofline_fraction_is_achieved_over_peak():
     assert r["frac"] == pytest.approx(1000.0 / 1377.3, abs=1e-4)
     r = bench.roofline("k", "hbm", 6.5514e9, 1.0e-3, pk, "GB/s")  # 6.55 GB in 1 ms = the measured peak
     assert r["frac"] == pytest.approx(1.0, abs=1e-4)
+
+
+def test_clock_summary_reads_nvidia_smi_samples():
+    """The clock record of a timed region: median SM clock over loaded samples (idle ones at the start or end are
+    left out), the maximum clock, and every throttle reason that was active in any sample; malformed lines are
+    skipped."""
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 345, 1965, 120.5, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",  # idle
+        "0, 1620, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1635, 1965, 1001.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1650, 1965, 990.7, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "[N/A], garbage",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = cs.summary()
+    assert s == {"sm_mhz": 1635.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 4}
+    cs.lines.append("0, 1500, 1965, 900.0, 0x0000000000000040, Not Active, Active, Not Active, Not Active")
+    assert bench.ClockSampler.summary(cs)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    empty = bench.ClockSampler(0)
+    assert empty.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
