@@ -73,3 +73,16 @@ def test_clock_summary_reads_nvidia_smi_samples():
     assert bench.ClockSampler.summary(cs)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     empty = bench.ClockSampler(0)
     assert empty.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_traffic_counters_only_for_the_captured_kernels(monkeypatch):
+    """roofline.traffic comes from the committed counter summary only while the kernel sources hash to the value
+    recorded with it, and only for the workload it was captured on."""
+    import json
+    with open(os.path.join(ROOT, "profiles", "traffic_hunyuan720.json")) as f:
+        rec = json.load(f)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["source_hash"])
+    assert bench.measured_traffic(rec["workload"])["sparse_attn"] == rec["sparse_attn"]
+    assert bench.measured_traffic("some-other-layer") == {}
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.measured_traffic(rec["workload"]) == {}
