@@ -4,7 +4,7 @@
 One step = the whole hot path over one synthetic attention layer: losa_dense_profile (dense forward + exact block
 masses), losa_select (tau = 0.99 by default) and losa_sparse_attn over the frozen lists. The default workload is the
 HunyuanVideo-720p-shaped layer (24 heads, 33x45x80 token grid, N = 118800 padded to 118912, head_dim 128, bf16,
-128 x 128 blocks), the layer the sparse-attention throughput target is quoted on.
+128 x 128 blocks).
 
 Prints ONE JSON line (rank 0). `value` is the dense-equivalent throughput of losa_sparse_attn, 4*H*N^2*d / t_sparse,
 summed over ranks (weak scaling: every rank runs its own layer); the per-kernel times, the profile+select time, the
