@@ -42,7 +42,7 @@ extern "C" {
 typedef enum {
     LOSA_OK = 0,
     LOSA_ERR_INVALID_ARG = -1,   /* null / misaligned pointer, inconsistent shape, tau outside (0, 1]      */
-    LOSA_ERR_UNSUPPORTED = -2,   /* a valid shape this build has no kernel for                          */
+    LOSA_ERR_UNSUPPORTED = -2,   /* a valid shape the library has no kernel for                         */
     LOSA_ERR_CAPACITY = -3,      /* an output or workspace buffer is smaller than the worst case          */
     LOSA_ERR_CUDA = -4,          /* the CUDA runtime reported an error at launch or synchronisation      */
     LOSA_ERR_DEVICE_FAULT = -5,  /* a kernel detected invalid data (bad block index, non-finite mass)   */
