@@ -229,7 +229,8 @@ class Drift:
         self.rms = []      # per layer: (3, H) fp32
         n = cfg.n_tokens
         for layer in layers:
-            ts = tuple(torch.from_numpy(layer.all_f32(name)).to(device) for name in ("q", "k", "v"))
+            # own copies: the walk must not write into the layer's arrays (a same-device .to() would alias them)
+            ts = tuple(torch.from_numpy(layer.all_f32(name)).to(device, copy=True) for name in ("q", "k", "v"))
             self.master.append(ts)
             self.rms.append(torch.stack([t[:, :n].pow(2).mean(dim=(1, 2)).sqrt() for t in ts]))
 

@@ -525,7 +525,45 @@ def test_generator_is_seeded_and_padded():
     np.testing.assert_array_equal(a.k, b.k)
     cfg = CONFIGS["tiny"]
     assert a.q.shape == (cfg.heads, cfg.n_padded, cfg.head_dim)
-    # config 1 geometry: 21*30*52 = 32760 tokens, padded to 32768 with zero rows
+    # Wan2.1-1.3B-480p geometry: 21*30*52 = 32760 tokens, padded to 32768 with zero rows
     c1 = CONFIGS["wan1.3b480"]
     assert (c1.n_tokens, c1.n_padded, c1.n_blocks) == (32760, 32768, 256)
     assert CONFIGS["hunyuan720"].n_padded == 118912 and CONFIGS["wan14b720"].n_padded == 75648
+
+
+def test_sample_items_is_seeded_and_keeps_the_forced_items():
+    """Sampled items are distinct, sorted, in range, reproducible from the seed, and always include the tail query
+    block of head 0 and the requested ids."""
+    from losa_synth import sample_items
+    cfg = CONFIGS["hunyuan720"]
+    total = cfg.heads * cfg.n_blocks
+    a = sample_items(cfg, 64, seed=3, must_include=[5, 700])
+    assert len(a) == 64 and len(set(a.tolist())) == 64 and (np.diff(a) > 0).all()
+    assert a.min() >= 0 and a.max() < total
+    assert {cfg.n_blocks - 1, 5, 700} <= set(a.tolist())
+    np.testing.assert_array_equal(a, sample_items(cfg, 64, seed=3, must_include=[5, 700]))
+    assert not np.array_equal(a, sample_items(cfg, 64, seed=4, must_include=[5, 700]))
+    small = CONFIGS["tiny"]
+    np.testing.assert_array_equal(sample_items(small, 1000), np.arange(small.heads * small.n_blocks))
+
+
+def test_drift_walk_on_the_host():
+    """The reuse loop's drift: each step adds amount * rms(step-0 head) * N(0, 1) to the real rows only, padded rows
+    stay zero, and the walk is reproducible from its seed."""
+    from losa_synth import Drift
+    cfg = CONFIGS["tiny"]
+    layer = make_layer(cfg)
+    d1 = Drift(cfg, [layer], device="cpu", amount=0.1, seed=7)
+    d2 = Drift(cfg, [layer], device="cpu", amount=0.1, seed=7)
+    q0 = d1.tokens(0)[0].clone()
+    d1.advance()
+    d2.advance()
+    q1 = d1.tokens(0)[0]
+    torch.testing.assert_close(q1, d2.tokens(0)[0], rtol=0, atol=0)
+    n = cfg.n_tokens
+    assert torch.count_nonzero(q1[:, n:]) == 0
+    step = (q1 - q0)[:, :n]
+    rms0 = q0[:, :n].pow(2).mean(dim=(1, 2)).sqrt()
+    ratio = step.pow(2).mean(dim=(1, 2)).sqrt() / (0.1 * rms0)
+    assert torch.allclose(ratio, torch.ones_like(ratio), atol=0.05), ratio
+    np.testing.assert_array_equal(layer.q, make_layer(cfg).q)  # the walk leaves the generated layer untouched
