@@ -36,16 +36,22 @@ METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select 
 KERNELS_PER_STEP = {"dense_profile": 1, "select": 3, "sparse_attn": 1}
 
 
-def peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            p = json.load(f)
-        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
-                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "sm_max_mhz": p.get("sm_max_mhz", 1965.0),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
-            "source": "fallback"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def peaks(path=None):
+    """Roofline denominators: the measured copy bandwidth and bf16 GEMM rates of this GPU model when the measurement
+    file is present (any missing entry falls back to the earlier measurement, and the source says so), else the
+    earlier measurement."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(path):
+        return {**FALLBACK_PEAKS, "source": "fallback"}
+    with open(path) as f:
+        p = json.load(f)
+    out = {k: float(p[k]) if isinstance(p.get(k), (int, float)) else v for k, v in FALLBACK_PEAKS.items()}
+    missing = [k for k in FALLBACK_PEAKS if not isinstance(p.get(k), (int, float))]
+    out["source"] = "measured" if not missing else "measured, fallback for " + ", ".join(missing)
+    return out
 
 
 def bench_config(cfg, tau, world):

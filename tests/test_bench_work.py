@@ -86,3 +86,20 @@ def test_traffic_counters_only_for_the_captured_kernels(monkeypatch):
     assert bench.measured_traffic("some-other-layer") == {}
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.measured_traffic(rec["workload"]) == {}
+
+
+def test_peaks_fall_back_per_missing_entry(tmp_path):
+    """The roofline denominators come from the measurement file; an entry it lacks falls back alone, and the source
+    names it; without the file every entry is the earlier measurement."""
+    import json
+    full = {"hbm_gbs": 6551.4, "bf16_tflops": 1618.2, "bf16_tflops_sustained": 1377.3, "sm_max_mhz": 1965.0}
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps(full))
+    p = bench.peaks(str(f))
+    assert p["source"] == "measured" and p["bf16_tflops_sustained"] == 1377.3 and p["hbm_gbs"] == 6551.4
+    f.write_text(json.dumps({k: v for k, v in full.items() if k != "bf16_tflops_sustained"}))
+    p = bench.peaks(str(f))
+    assert p["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert p["hbm_gbs"] == 6551.4 and "fallback for bf16_tflops_sustained" in p["source"]
+    p = bench.peaks(str(tmp_path / "absent.json"))
+    assert p["source"] == "fallback" and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
