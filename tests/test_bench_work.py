@@ -103,3 +103,8 @@ def test_peaks_fall_back_per_missing_entry(tmp_path):
     assert p["hbm_gbs"] == 6551.4 and "fallback for bf16_tflops_sustained" in p["source"]
     p = bench.peaks(str(tmp_path / "absent.json"))
     assert p["source"] == "fallback" and p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+
+
+def test_l2_note_matches_the_workload_size():
+    assert bench.bench_config(CONFIGS["hunyuan720"], 0.99, 1)["l2"].startswith("inputs larger than L2")
+    assert bench.bench_config(CONFIGS["tiny"], 0.99, 1)["l2"].startswith("inputs fit in L2")
