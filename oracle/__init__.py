@@ -1,6 +1,7 @@
 """ctypes wrapper of the fp64 CPU oracle (losa_oracle.cpp) — TEST INFRASTRUCTURE ONLY.
 
-Only the tests, `__graft_entry__.smoke()` and the benchmark's CPU-baseline leg may import this package.
+Only the tests, `__graft_entry__.smoke()` and the benchmark's two CPU legs (`cpu_baseline` and `--impl reference`)
+may import this package.
 It is independent of the CUDA library: it neither imports nor loads anything from it.
 """
 from __future__ import annotations

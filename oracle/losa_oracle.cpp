@@ -1,8 +1,8 @@
 // Oracle for the LoSA hot path — TEST INFRASTRUCTURE ONLY.
 //
 // A plain, slow, obviously-correct CPU implementation in fp64 of what the CUDA library computes. Only the
-// tests, the smoke check and the benchmark's CPU-baseline leg may load it. It shares no code, header, table
-// or constant with the CUDA path, and the product path never calls it.
+// tests, the smoke check and the benchmark's two CPU legs (its cpu_baseline and its reference arm) may load it.
+// It shares no code, header, table or constant with the CUDA path, and the product path never calls it.
 //
 // Source of every definition: the page "LoSA: Near-Lossless Sparse Attention for Training-Free Video
 // Diffusion Acceleration" (m.montaan.com/papers/2608.12032):
