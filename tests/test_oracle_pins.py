@@ -170,6 +170,27 @@ def test_mass_block_diagonal():
     np.testing.assert_allclose(m, np.eye(nb), atol=1e-20)
 
 
+def test_mass_ragged_tail_dominant_keys():
+    """Real query r sees one key perm[r] with a logit 100 above all others, so A(r, .) is that key up to e^-100:
+    M(i, j) = (real rows of block i whose key lies in block j) / R_i, also for the ragged tail block, whose zero
+    padded query rows must not count."""
+    N, Np, R, C = 100, 128, 32, 16
+    rng = np.random.default_rng(17)
+    perm = rng.permutation(N)
+    q = np.zeros((1, Np, N), np.float32)
+    k = np.zeros((1, Np, N), np.float32)
+    for r in range(N):
+        q[0, r, r] = 10.0
+        k[0, perm[r], r] = 10.0
+    import oracle
+    m = oracle.mass(q, k, N, R, C, 1.0)
+    want = np.zeros((Np // R, Np // C))
+    for r in range(N):
+        want[r // R, perm[r] // C] += 1.0
+    want /= np.array([min(R, N - i * R) for i in range(Np // R)], np.float64)[:, None]
+    np.testing.assert_allclose(m, want, atol=1e-30)
+
+
 def test_mass_from_library_attention_probabilities():
     """A is recovered from the library's attention with V = identity (O = A I = A); block sums of A,
     divided by the real rows, must equal the oracle's M. Uneven R != C and a ragged tail."""
