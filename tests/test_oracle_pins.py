@@ -588,3 +588,41 @@ def test_drift_walk_on_the_host():
     ratio = step.pow(2).mean(dim=(1, 2)).sqrt() / (0.1 * rms0)
     assert torch.allclose(ratio, torch.ones_like(ratio), atol=0.05), ratio
     np.testing.assert_array_equal(layer.q, make_layer(cfg).q)  # the walk leaves the generated layer untouched
+
+
+def test_lpt_order_invariants():
+    """The work order is a permutation along which list lengths never increase, and items of equal length appear in
+    increasing id order (many ties)."""
+    rng = np.random.default_rng(18)
+    import oracle
+    for n in (1, 2, 7, 300):
+        counts = rng.integers(1, 4, n).astype(np.int32)
+        order = oracle.lpt_order(counts)
+        assert sorted(order.tolist()) == list(range(n))
+        c = counts[order]
+        assert (np.diff(c) <= 0).all()
+        for v in np.unique(c):
+            ids = order[c == v]
+            assert (np.diff(ids) > 0).all()
+
+
+def test_select_topk_boundary_invariants():
+    """Top-k keeps min(k, nk) blocks, every kept mass is at least every dropped one, and where equal masses straddle
+    the cut the kept ones have the lower indices."""
+    rng = np.random.default_rng(19)
+    import oracle
+    for trial in range(200):
+        nk = int(rng.integers(1, 30))
+        m = rng.integers(0, 4, nk).astype(np.float32)  # many ties
+        k = int(rng.integers(1, nk + 2))
+        counts, idx = oracle.select_topk(m[None], k)
+        kept = set(idx[0, :counts[0]].tolist())
+        assert counts[0] == min(k, nk) and len(kept) == counts[0]
+        dropped = [j for j in range(nk) if j not in kept]
+        if dropped and kept:
+            assert min(m[j] for j in kept) >= max(m[j] for j in dropped)
+            cut = min(m[j] for j in kept)
+            tied_kept = [j for j in kept if m[j] == cut]
+            tied_dropped = [j for j in dropped if m[j] == cut]
+            if tied_dropped:
+                assert max(tied_kept) < min(tied_dropped)
