@@ -38,6 +38,19 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(raw, n), n
 
 
+def test_every_exported_symbol_is_declared(lib):
+    """The reverse direction: the library exports no losa_* entry point that the header does not declare (read from
+    the dynamic symbol table with nm; skipped where nm is missing)."""
+    import shutil
+    import subprocess
+    if not shutil.which("nm"):
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", L.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.split() and line.split()[-1].startswith("losa_")}
+    assert exported and exported <= _declared(), exported - _declared()
+
+
 def test_status_strings(lib):
     for code, name in L.STATUS.items():
         assert L.losa_status_string(code) == name
