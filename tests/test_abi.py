@@ -166,3 +166,41 @@ def test_binding_refuses_wrong_tensors_before_the_call(lib):
     with pytest.raises(ValueError, match="lse: expected torch.float32"):
         L.losa_sparse_attn(s, tok(), tok(), tok(), 0.1, i32(rows + 1), i32(1), None, tok(),
                            torch.empty(H * Np, dtype=torch.float64))
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "losa.h"
+int main(void) {
+    losa_shape good = {2, 1000, 1024, 128, 128, 128, LOSA_DTYPE_BF16};
+    losa_shape bad = good;
+    bad.n_padded = 1000;
+    if (losa_version() < 100) return 1;
+    if (strcmp(losa_status_string(LOSA_ERR_CAPACITY), "LOSA_ERR_CAPACITY") != 0) return 2;
+    if (losa_select_workspace_bytes(&good) == 0 || losa_select_workspace_bytes(&bad) != 0) return 3;
+    if (losa_dense_profile(&bad, 0, 0, 0, 0.1f, 0, 0, 0, 0) != LOSA_ERR_INVALID_ARG) return 4;
+    if (losa_sparse_attn(&good, 0, 0, 0, 0.1f, 0, 0, 0, 0, 0, 0) != LOSA_ERR_INVALID_ARG) return 5;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program that includes only include/losa.h, links liblosa.so and calls the
+    host-side entry points runs without Python or torch (none of these calls reaches the CUDA runtime)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if not gcc or not os.path.isdir(cuda_inc):
+        pytest.skip("gcc or the CUDA headers are not available")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(L.library_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src),
+                    "-L", libdir, "-llosa", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
