@@ -139,7 +139,8 @@ losa_status losa_select_noalloc(const losa_shape* shape, const float* mass, doub
  *   indptr, kv_block_idx : the CSR lists written by losa_select (any order within a row is accepted; every
  *                   index must lie in [0, nk), every row must be non-empty).
  *   order         : [H*nq] permutation of item ids giving the work order (longest list first for balance),
- *                   or NULL for ascending item order.
+ *                   or NULL for ascending item order. Its entries are not checked on the device: an entry outside
+ *                   [0, H*nq) is undefined behaviour (losa_select always writes a valid permutation).
  *   o             : [H][Np][d] output; lse: [H][Np] fp32 output or NULL.
  * An out-of-range block index or an empty row sets the device error word (LOSA_ERR_DEVICE_FAULT); the
  * affected rows are left unspecified.
