@@ -137,7 +137,9 @@ losa_status losa_select_noalloc(const losa_shape* shape, const float* mass, doub
  * those keys only).
  *   q, k, v       : [H][Np][d] tokens of the current step (they may differ from the profiled step's).
  *   indptr, kv_block_idx : the CSR lists written by losa_select (any order within a row is accepted; every
- *                   index must lie in [0, nk), every row must be non-empty).
+ *                   index must lie in [0, nk), every row must be non-empty). indptr must be non-decreasing, and
+ *                   its last entry must not exceed the length of kv_block_idx: the library cannot check the
+ *                   latter (it is not told that length), and a violation is undefined behaviour.
  *   order         : [H*nq] permutation of item ids giving the work order (longest list first for balance),
  *                   or NULL for ascending item order. Its entries are not checked on the device: an entry outside
  *                   [0, H*nq) is undefined behaviour (losa_select always writes a valid permutation).
