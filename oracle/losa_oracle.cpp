@@ -88,6 +88,11 @@ int select_row(const T* m, int nk, double tau, int32_t* out) {
     std::iota(ord.begin(), ord.end(), 0);
     for (int j = 0; j < nk; ++j)
         if (!(m[j] >= (T)0) || std::isinf((double)m[j])) return -1;
+    // Input domain: a row of block masses normalised to one (R2), with slack for rounding. A row summing to more than
+    // 2 is refused, which also keeps every unit below 2^53 and the row total far from 2^64.
+    double row_sum = 0.0;
+    for (int j = 0; j < nk; ++j) row_sum += (double)m[j];
+    if (row_sum > 2.0) return -1;
     // Decreasing mass, ties by ascending index (R3). Comparison on the stored value itself.
     std::sort(ord.begin(), ord.end(), [&](int a, int b) { return m[a] > m[b] || (m[a] == m[b] && a < b); });
     // Integer units u_j = ceil(M_j * 2^52): scaling by a power of two is exact in fp64, so is ceil.

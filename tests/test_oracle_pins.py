@@ -405,6 +405,29 @@ def test_select_rejects_bad_tau():
             oracle.select(m, tau)
 
 
+def test_select_refuses_rows_outside_the_normalised_domain():
+    """The selection reads rows of masses normalised to one (the LoSA page's "theta R" rule divided by R): a row
+    summing to more than 2 (here one scaled by 1e4, whose integer units would leave 64 bits) is refused, while a row
+    whose sum is one up to rounding, or a single block holding all the mass, is accepted."""
+    import oracle
+    rng = np.random.default_rng(13)
+    m = rng.exponential(size=(3, 50))
+    m /= m.sum(axis=1, keepdims=True)
+    for dt in (np.float64, np.float32):
+        oracle.select(m.astype(dt), 0.99)
+        big = m.copy()
+        big[1] *= 1e4
+        with pytest.raises(ValueError):
+            oracle.select(big.astype(dt), 0.99)
+        one = np.zeros((1, 5), dt)
+        one[0, 3] = 1.0
+        counts, idx = oracle.select(one, 0.99)
+        assert counts[0] == 1 and idx[0, 0] == 3
+        over = np.full((1, 4), 0.5000001, dt)  # sums to 2.0000004
+        with pytest.raises(ValueError):
+            oracle.select(over, 0.5)
+
+
 def test_lpt_order_definition():
     rng = np.random.default_rng(10)
     import oracle
