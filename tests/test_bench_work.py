@@ -50,6 +50,10 @@ def test_roofline_fraction_is_achieved_over_peak():
     r = bench.roofline("k", "tensor", 2.0e12, 2.0e-3, pk, "TFLOP/s")  # 2e12 flop in 2 ms = 1000 TFLOP/s
     assert r["achieved"] == pytest.approx(1000.0)
     assert r["frac"] == pytest.approx(1000.0 / 1377.3, abs=1e-4)
+    assert r["frac_of_burst"] == pytest.approx(1000.0 / 1618.0, abs=1e-4)
+    assert r["frac_of_sustained"] == pytest.approx(r["frac"])
+    r = bench.roofline("k", "tensor", 2.0e12, 2.0e-3, pk, "TFLOP/s", peak_kind="burst")
+    assert r["frac"] == pytest.approx(1000.0 / 1618.0, abs=1e-4) and r["peak"] == 1618.0
     r = bench.roofline("k", "hbm", 6.5514e9, 1.0e-3, pk, "GB/s")  # 6.55 GB in 1 ms = the measured peak
     assert r["frac"] == pytest.approx(1.0, abs=1e-4)
 
