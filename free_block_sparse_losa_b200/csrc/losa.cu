@@ -32,8 +32,8 @@ namespace {
 
 unsigned long long g_wait_limit_ns = 2000000000ull;
 
-constexpr int kMaxSelectItems = 32768;   // longest-first order is sorted by one CTA in shared memory
-constexpr int kMaxSelectBlocks = 8192;   // per-row sort in shared memory
+constexpr long long kMaxSelectItems = 1ll << 20;  // (head, query block) rows per selection call
+constexpr int kMaxSelectBlocks = 8192;            // per-row sort in shared memory
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -226,17 +226,68 @@ int next_pow2(int n) {
     return p;
 }
 
-// Kernel 1 of the selection: the warp-per-row register form for nk <= 1024, else the CTA shared-memory form.
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace of the selection calls: per-row staged lists and counts, then the order kernels' per-chunk histograms,
+// chunk offsets and completion counter. Every region starts on a 256-byte boundary.
+struct SelectLayout {
+    size_t staged, counts, table, chunk_off, ticket, total;
+    int nch;
+};
+
+SelectLayout select_layout(long long rows, int nk) {
+    SelectLayout L;
+    L.nch = (int)((rows + kOrderChunk - 1) / kOrderChunk);
+    size_t off = 0;
+    L.staged = off;
+    off += align256((size_t)rows * nk * sizeof(int32_t));
+    L.counts = off;
+    off += align256((size_t)rows * sizeof(int32_t));
+    L.table = off;
+    off += align256((size_t)nk * L.nch * sizeof(int32_t));
+    L.chunk_off = off;
+    off += align256((size_t)L.nch * sizeof(int64_t));
+    L.ticket = off;
+    off += 256;
+    L.total = off;
+    return L;
+}
+
+size_t select_ws_bytes(const losa_shape* s) {
+    const long long rows = (long long)s->heads * (s->n_padded / s->block_q);
+    return select_layout(rows, s->n_padded / s->block_k).total;
+}
+
+// Kernel 1: the pick path, one warp per row (in registers for nk <= 1024, in shared memory above), then a full sort
+// of the rows it leaves undecided (one warp per row in registers, or one CTA per row in shared memory).
 losa_status launch_select_rows(const float* mass, int nk, int rows, double tau, int topk, int32_t* counts,
-                               int32_t* staged, cudaStream_t stream) {
+                               int32_t* staged, uint32_t* ticket, cudaStream_t stream) {
     const unsigned wgrid = (unsigned)((rows + 7) / 8);
-    if (nk <= 32) select_rows_warp_kernel<1><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
-    else if (nk <= 64) select_rows_warp_kernel<2><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
-    else if (nk <= 128) select_rows_warp_kernel<4><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
-    else if (nk <= 256) select_rows_warp_kernel<8><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
-    else if (nk <= 512) select_rows_warp_kernel<16><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
-    else if (nk <= 1024) select_rows_warp_kernel<32><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);
+#define LOSA_ROWS_WARP(E)                                                                                        \
+    do {                                                                                                         \
+        select_pick_warp_kernel<E><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged, ticket); \
+        const losa_status st1 = launch_status();                                                                 \
+        if (st1 != LOSA_OK) return st1;                                                                          \
+        select_sort_warp_kernel<E><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);       \
+    } while (0)
+    if (nk <= 32) LOSA_ROWS_WARP(1);
+    else if (nk <= 64) LOSA_ROWS_WARP(2);
+    else if (nk <= 128) LOSA_ROWS_WARP(4);
+    else if (nk <= 256) LOSA_ROWS_WARP(8);
+    else if (nk <= 512) LOSA_ROWS_WARP(16);
+    else if (nk <= 1024) LOSA_ROWS_WARP(32);
+#undef LOSA_ROWS_WARP
     else {
+        int wpc = (int)(65536 / ((size_t)nk * sizeof(uint32_t)));  // rows (warps) per CTA: at most 64 KB of rows
+        wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+        const size_t smem = (size_t)wpc * nk * sizeof(uint32_t);
+        if (cudaFuncSetAttribute(select_pick_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return LOSA_ERR_CUDA;
+        select_pick_smem_kernel<<<(unsigned)((rows + wpc - 1) / wpc), (unsigned)(32 * wpc), smem, stream>>>(
+            mass, nk, rows, tau, topk, counts, staged, ticket);
+        losa_status st = launch_status();
+        if (st != LOSA_OK) return st;
         const int n2 = next_pow2(nk);
         const size_t smem1 = (size_t)n2 * sizeof(uint64_t) + (size_t)nk;
         if (cudaFuncSetAttribute(select_rows_kernel<kSelectThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -248,12 +299,51 @@ losa_status launch_select_rows(const float* mass, int nk, int rows, double tau, 
     return launch_status();
 }
 
-size_t select_ws_bytes(const losa_shape* s) {
-    const size_t rows = (size_t)s->heads * (s->n_padded / s->block_q);
-    const size_t nk = (size_t)(s->n_padded / s->block_k);
-    const size_t staged = (rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
-    const size_t counts = (rows * sizeof(int32_t) + 255) & ~(size_t)255;
-    return staged + counts;
+// The selection shared by losa_select, losa_select_topk and losa_select_noalloc: argument checks, then the
+// stream-ordered launches (the rows' cut in two kernels, histograms, order and indptr, scatter). topk > 0 selects a fixed count instead of
+// the mass threshold tau. ws is the workspace (at least select_ws_bytes); ws_bytes is its size.
+losa_status run_select(const losa_shape* shape, const float* mass, double tau, int topk, int32_t* indptr,
+                       int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (topk == 0 && !(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_INVALID_ARG;
+    if (topk < 0) return LOSA_ERR_INVALID_ARG;
+    if (!aligned16(mass) || !indptr || !kv_block_idx || !order || !aligned16(ws)) return LOSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
+         reinterpret_cast<uintptr_t>(order)) & 3u)
+        return LOSA_ERR_INVALID_ARG;
+    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
+    const long long rows = (long long)shape->heads * nq;
+    // indptr is int32: every row's list, even at its longest, must fit
+    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks || rows * nk > 2147483647ll) return LOSA_ERR_UNSUPPORTED;
+    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
+    const SelectLayout lay = select_layout(rows, nk);
+    if (ws_bytes < lay.total) return LOSA_ERR_CAPACITY;
+
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* staged = reinterpret_cast<int32_t*>(w + lay.staged);
+    int32_t* counts = reinterpret_cast<int32_t*>(w + lay.counts);
+    int32_t* table = reinterpret_cast<int32_t*>(w + lay.table);
+    int64_t* chunk_off = reinterpret_cast<int64_t*>(w + lay.chunk_off);
+    uint32_t* ticket = reinterpret_cast<uint32_t*>(w + lay.ticket);
+
+    if ((st = launch_select_rows(mass, nk, (int)rows, topk ? 1.0 : tau, topk, counts, staged, ticket, stream)) !=
+        LOSA_OK)
+        return st;
+    const size_t hsmem = (size_t)nk * sizeof(int32_t);  // <= 32 KB, beside the kernel's 32 KB scan segment
+    if (cudaFuncSetAttribute(select_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem) !=
+        cudaSuccess)
+        return LOSA_ERR_CUDA;
+    select_hist_kernel<<<(unsigned)lay.nch, kOrderChunk, hsmem, stream>>>(counts, (int)rows, nk, lay.nch, table,
+                                                                          chunk_off, ticket, indptr);
+    if ((st = launch_status()) != LOSA_OK) return st;
+    select_order_kernel<<<(unsigned)lay.nch, kOrderChunk, hsmem, stream>>>(counts, (int)rows, nk, lay.nch, table,
+                                                                           chunk_off, indptr, order);
+    if ((st = launch_status()) != LOSA_OK) return st;
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
+    return launch_status();
 }
 
 }  // namespace
@@ -305,67 +395,15 @@ size_t losa_select_workspace_bytes(const losa_shape* shape) {
 losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
                         int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
                         size_t ws_bytes, cudaStream_t stream) {
-    losa_status st = check_shape(shape);
-    if (st != LOSA_OK) return st;
-    if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_INVALID_ARG;
-    if (!aligned16(mass) || !indptr || !kv_block_idx || !order || !aligned16(workspace)) return LOSA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
-         reinterpret_cast<uintptr_t>(order)) & 3u)
-        return LOSA_ERR_INVALID_ARG;
-    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
-    const long long rows = (long long)shape->heads * nq;
-    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
-    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
-    if (ws_bytes < select_ws_bytes(shape)) return LOSA_ERR_CAPACITY;
-
-    int32_t* staged = static_cast<int32_t*>(workspace);
-    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
-    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
-
-    if ((st = launch_select_rows(mass, nk, (int)rows, tau, 0, counts, staged, stream)) != LOSA_OK) return st;
-
-    const int r2 = next_pow2((int)rows);
-    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
-    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem2) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
-    if ((st = launch_status()) != LOSA_OK) return st;
-
-    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
-    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
-    return launch_status();
+    return run_select(shape, mass, tau, 0, indptr, kv_block_idx, idx_capacity, order, workspace, ws_bytes, stream);
 }
 
 losa_status losa_select_topk(const losa_shape* shape, const float* mass, int32_t k_blocks, int32_t* indptr,
                              int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
                              size_t ws_bytes, cudaStream_t stream) {
-    losa_status st = check_shape(shape);
-    if (st != LOSA_OK) return st;
     if (k_blocks < 1) return LOSA_ERR_INVALID_ARG;
-    if (!aligned16(mass) || !indptr || !kv_block_idx || !order || !aligned16(workspace)) return LOSA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
-         reinterpret_cast<uintptr_t>(order)) & 3u)
-        return LOSA_ERR_INVALID_ARG;
-    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
-    const long long rows = (long long)shape->heads * nq;
-    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
-    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
-    if (ws_bytes < select_ws_bytes(shape)) return LOSA_ERR_CAPACITY;
-    int32_t* staged = static_cast<int32_t*>(workspace);
-    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
-    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + staged_bytes);
-    if ((st = launch_select_rows(mass, nk, (int)rows, 1.0, k_blocks, counts, staged, stream)) != LOSA_OK) return st;
-    const int r2 = next_pow2((int)rows);
-    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
-    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem2) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
-    if ((st = launch_status()) != LOSA_OK) return st;
-    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
-    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
-    return launch_status();
+    return run_select(shape, mass, 1.0, k_blocks, indptr, kv_block_idx, idx_capacity, order, workspace, ws_bytes,
+                      stream);
 }
 
 losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
@@ -374,6 +412,9 @@ losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void*
     losa_status st = check_shape(shape);
     if (st != LOSA_OK) return st;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !indptr || !kv_block_idx)
+        return LOSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
+         reinterpret_cast<uintptr_t>(order)) & 3u)  // int32 arrays (order may be NULL)
         return LOSA_ERR_INVALID_ARG;
     if (lse && !aligned16(lse)) return LOSA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
@@ -424,9 +465,10 @@ extern "C" losa_status losa_selftest_wait_timeout(uint32_t limit_ns, cudaStream_
 // Some callers cannot allocate device memory at call time: a serving process that reserved nearly all of the GPU's
 // memory for its own pool at start-up (a cudaMalloc then fails or would bypass its accounting), a plugin whose host
 // framework owns every buffer and offers no workspace, or a latency-critical path where cudaMalloc / cudaFree may
-// synchronise the device. losa_select_noalloc serves them: it runs the same three selection kernels as losa_select,
-// but their scratch (the per-row staging lists and the per-row counts) lives in the fixed device array below, which
-// every GPU that loads this library holds until the process exits.
+// synchronise the device. losa_select_noalloc serves them: it runs the same selection kernels as losa_select, but
+// their scratch (the per-row staging lists and counts, the order kernels' histograms, chunk offsets and completion
+// counter) lives in the fixed device array below, which every GPU that loads this library holds until the process
+// exits.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
@@ -435,20 +477,48 @@ static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchB
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read). A device reset ends the primary context;
+// the next one gets a new id, and the library's device code (with the array) is loaded again at a new address.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 // Device address of g_select_scratch on the current device. In host code the array's name only stands in for the
-// symbol; the address a kernel can use comes from cudaGetSymbolAddress, looked up once per device with that device
-// current (the lookup may load this library's device code onto the device).
+// symbol; the address a kernel can use comes from cudaGetSymbolAddress, looked up with that device current, once per
+// device and context (the lookup may load this library's device code onto the device).
 void* scratch_on_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = p;
-    }
-    return g_scratch_ptr[dev];
+    const unsigned long long ctx = current_context_id();
+    if (g_scratch_ptr[dev] && ctx != 0 && g_scratch_ctx[dev] == ctx) return g_scratch_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();  // the lookup has made the device's context current
+    return p;
 }
 
 }  // namespace
@@ -458,35 +528,12 @@ extern "C" losa_status losa_select_noalloc(const losa_shape* shape, const float*
                                            cudaStream_t stream) {
     losa_status st = check_shape(shape);
     if (st != LOSA_OK) return st;
-    if (!(tau > 0.0 && tau <= 1.0)) return LOSA_ERR_INVALID_ARG;
-    if (!aligned16(mass) || !indptr || !kv_block_idx || !order) return LOSA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(indptr) | reinterpret_cast<uintptr_t>(kv_block_idx) |
-         reinterpret_cast<uintptr_t>(order)) & 3u)
-        return LOSA_ERR_INVALID_ARG;
-    const int nq = shape->n_padded / shape->block_q, nk = shape->n_padded / shape->block_k;
-    const long long rows = (long long)shape->heads * nq;
-    if (rows > kMaxSelectItems || nk > kMaxSelectBlocks) return LOSA_ERR_UNSUPPORTED;
-    if (idx_capacity < rows * nk) return LOSA_ERR_CAPACITY;
-    // The fixed scratch must hold rows * nk staged indices plus rows counts.
+    // The fixed scratch must hold every region of the selection's workspace for this shape.
     if (select_ws_bytes(shape) > kNoAllocScratchBytes) return LOSA_ERR_CAPACITY;
-
     void* scratch = scratch_on_current_device();
     if (!scratch) return LOSA_ERR_CUDA;
-    // Both scratch regions are fully written before they are read, so stale contents from an earlier call need
-    // no clearing.
-    int32_t* staged = static_cast<int32_t*>(scratch);
-    const size_t staged_bytes = ((size_t)rows * nk * sizeof(int32_t) + 255) & ~(size_t)255;
-    int32_t* counts = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(scratch) + staged_bytes);
-
-    if ((st = launch_select_rows(mass, nk, (int)rows, tau, 0, counts, staged, stream)) != LOSA_OK) return st;
-    const int r2 = next_pow2((int)rows);
-    const size_t smem2 = (size_t)r2 * sizeof(uint32_t);
-    if (cudaFuncSetAttribute(select_finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem2) != cudaSuccess)
-        return LOSA_ERR_CUDA;
-    select_finalize_kernel<1024><<<1, 1024, smem2, stream>>>(counts, (int)rows, nk, r2, indptr, order);
-    if ((st = launch_status()) != LOSA_OK) return st;
-    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
-    select_scatter_kernel<<<blocks, 256, 0, stream>>>(staged, counts, indptr, (int)rows, nk, kv_block_idx);
-    return launch_status();
+    // Regions are written before they are read; the one counter that must start at zero is cleared by the call's
+    // first kernel. Stale contents from an earlier call need no other clearing.
+    return run_select(shape, mass, tau, 0, indptr, kv_block_idx, idx_capacity, order, scratch, kNoAllocScratchBytes,
+                      stream);
 }

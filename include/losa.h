@@ -25,8 +25,8 @@
  * Supported shapes: dtype BF16 with head_dim 128, block_q = 128 and block_k = 128 or 32 (tensor-core path; 32 is the
  * LoSA page's key-block size), or dtype F32 with head_dim 64 or 128 and block_q = block_k in {32, 64, 128} (exact fp32
  * path for small checks). Size limits: the tensor-core path takes Np <= 131072 (1024 blocks of 128 tokens per head);
- * the selection calls take nk <= 8192 key blocks per row and H * nq <= 32768 items per call. Any other valid shape
- * returns LOSA_ERR_UNSUPPORTED before anything is launched.
+ * the selection calls take nk <= 8192 key blocks per row, H * nq <= 1048576 items per call and H * nq * nk < 2^31
+ * (the CSR offsets are int32). Any other valid shape returns LOSA_ERR_UNSUPPORTED before anything is launched.
  */
 #ifndef LOSA_H
 #define LOSA_H
@@ -82,20 +82,24 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
  * Mass-threshold selection (LoSA page, Methodology Summary, "One-time pattern construction": sort the key
  * blocks of one (head, query block) by decreasing mass and keep the shortest prefix whose mass reaches
  * theta times the block's total).
- *   mass          : [H][nq][nk] fp32, non-negative, finite (as written by losa_dense_profile).
+ *   mass          : [H][nq][nk] fp32 rows normalised to one, as losa_dense_profile writes them: every entry finite
+ *                   and >= 0, every row summing to at most 2 (the slack covers rounding).
  *   tau           : retained-mass threshold in (0, 1].
  *   indptr        : [H*nq + 1] int32 output; row r's kept blocks are kv_block_idx[indptr[r] .. indptr[r+1]).
  *                   indptr[H*nq] = nnz stays on the device; reading it back is the caller's choice.
  *   kv_block_idx  : [idx_capacity] int32 output, kept key-block indices of each row in ascending order.
  *   idx_capacity  : must be >= H*nq*nk (the worst case), else LOSA_ERR_CAPACITY.
  *   order         : [H*nq] int32 output, item ids by list length descending, ties by ascending id (the
- *                   longest-first work order losa_sparse_attn consumes). At most 32768 items per call.
+ *                   longest-first work order losa_sparse_attn consumes).
  *   workspace     : device scratch of at least losa_select_workspace_bytes(shape) bytes (16-byte aligned);
  *                   its contents on entry do not matter.
  * Rule per row: order blocks by (mass descending, index ascending); u_j = ceil(M_j * 2^52) as 64-bit integers;
  * T = ceil(tau * sum_j u_j) in IEEE double; keep the first s >= 1 blocks whose integer prefix reaches T. The
  * integer prefix makes the result independent of summation order, and tau = 1 keeps exactly the non-zero blocks.
- * A negative or non-finite mass sets the device error word (LOSA_ERR_DEVICE_FAULT) and is treated as zero.
+ * A negative or non-finite mass sets the device error word (LOSA_ERR_DEVICE_FAULT) and is treated as zero. A row
+ * summing to more than 2 sets it too, and that row's list is unspecified (units are formed from min(M_j, 2), so
+ * nothing overflows and no arithmetic is undefined). Four stream-ordered launches: the per-row cut, per-chunk histograms of the list
+ * lengths, indptr with the work order, and the copy of the lists into place.
  */
 losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
                         int32_t* kv_block_idx, int64_t idx_capacity, int32_t* order, void* workspace,
@@ -123,8 +127,10 @@ size_t losa_select_workspace_bytes(const losa_shape* shape);
  *   Scratch: a fixed 16 MiB device array inside the library, present on every GPU that loads it until the process
  *   exits. Shapes whose scratch need (losa_select_workspace_bytes) exceeds 16 MiB return LOSA_ERR_CAPACITY: that
  *   admits H * nq * nk up to about 4.1 million (a 12-head layer of 256 x 256 blocks needs 3.2 MB).
- *   The library allocates nothing in this call. Its first call on a device looks up the array's device address
- *   (which may load the library's device code onto that device), so make that first call before any stream capture.
+ *   The library allocates nothing in this call. Its first call on a device (and the first after a device reset, which
+ *   loads the library's device code again) looks up the array's device address, which may load the library's device
+ *   code onto that device, so make that first call before any stream capture. The call's first kernel clears the one
+ *   counter in the array that must start at zero.
  *   Every call on a device shares the one array and overwrites what the previous call left there: calls whose GPU
  *   work can overlap (different streams without ordering between them) race on it and must be serialised.
  */

@@ -88,6 +88,9 @@ def test_pointer_and_tau_validation(lib):
     assert L.losa_dense_profile(s, FAKE, FAKE, FAKE, 0.1, FAKE, None, FAKE, stream=0, raise_on_error=False) == -1
     assert L.losa_dense_profile(s, FAKE, FAKE, FAKE, float("nan"), FAKE, FAKE, None, stream=0,
                                 raise_on_error=False) == -1
+    # the sparse call's int32 arrays must be 4-byte aligned (order may be NULL)
+    for ip, kv, od in ((FAKE + 2, FAKE, None), (FAKE, FAKE + 1, None), (FAKE, FAKE, FAKE + 2)):
+        assert L.losa_sparse_attn(s, FAKE, FAKE, FAKE, 0.1, ip, kv, od, FAKE, stream=0, raise_on_error=False) == -1
     ws = L.losa_select_workspace_bytes(s)
     for tau in (0.0, -1.0, 1.5, float("nan")):
         assert L.losa_select(s, FAKE, tau, FAKE, FAKE, FAKE, FAKE, idx_capacity=2 * 8 * 8, ws_bytes=ws, stream=0,
@@ -115,11 +118,18 @@ def test_capacity_and_unsupported(lib):
     wide = L.make_shape(1, 262200, 262272, 128, 128, 32, "bf16")
     assert L.losa_select(wide, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40,
                          ws_bytes=L.losa_select_workspace_bytes(wide), stream=0, raise_on_error=False) == -2
-    # more items than one selection call orders
-    big = L.make_shape(300, 130000, 130048, 128, 128, 128, "bf16")
-    wsb = L.losa_select_workspace_bytes(big)
-    assert L.losa_select(big, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40, ws_bytes=wsb, stream=0,
-                         raise_on_error=False) == -2
+    # more than 2^20 items in one selection call, and lists whose offsets could leave int32
+    for big in (L.make_shape(1100, 130000, 130048, 128, 128, 128, "bf16"),
+                L.make_shape(600, 131000, 131072, 128, 128, 32, "bf16")):
+        wsb = L.losa_select_workspace_bytes(big)
+        assert L.losa_select(big, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40, ws_bytes=wsb, stream=0,
+                             raise_on_error=False) == -2
+    # two guidance branches at the HunyuanVideo shape (44592 items) are supported: the call gets as far as the
+    # workspace check, which comes after the size limits (one byte short, so nothing is launched)
+    cfg2 = L.make_shape(48, 118800, 118912, 128, 128, 128, "bf16")
+    wsb = L.losa_select_workspace_bytes(cfg2)
+    assert L.losa_select(cfg2, FAKE, 0.99, FAKE, FAKE, FAKE, FAKE, idx_capacity=1 << 40, ws_bytes=wsb - 1, stream=0,
+                         raise_on_error=False) == -3
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):

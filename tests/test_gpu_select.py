@@ -76,7 +76,48 @@ def test_select_full_size_hunyuan_rows(oracle_mod):
     _run((H, nb, nb, 128, 128), m, 0.99, oracle_mod)
 
 
-@pytest.mark.parametrize("H,nb,k", [(1, 1, 1), (2, 31, 4), (4, 256, 12), (1, 929, 40), (2, 64, 64), (2, 64, 100)])
+def test_select_two_branch_hunyuan_rows(oracle_mod):
+    """Classifier-free guidance at the HunyuanVideo-720p shape: the conditional and unconditional branches stacked as
+    48 heads, 44592 rows x 929 blocks, each branch with its own pattern (LoSA page, Methodology Summary)."""
+    rng = np.random.default_rng(5)
+    H, nb = 48, 929
+    m = _masses(rng, H * nb, nb, "peaked")
+    counts = _run((H, nb, nb, 128, 128), m, 0.99, oracle_mod)
+    assert counts.min() >= 1
+
+
+@pytest.mark.parametrize("kind", ["exp", "ties", "peaked", "uniform"])
+def test_select_wide_rows_c32(kind, oracle_mod):
+    """3716 key blocks per row (the HunyuanVideo shape with 32-key blocks): the shared-memory pick path, and the
+    one-CTA sort for rows whose cut lies beyond the pick path's reach (uniform rows, tau = 1)."""
+    rng = np.random.default_rng(6)
+    H, nk = 1, 3716
+    nq = nk * 32 // 128  # 929 query blocks of 128 rows
+    m = _masses(rng, H * nq, nk, kind)
+    for tau in (0.9, 0.99, 1.0):
+        _run((H, nq, nk, 128, 32), m, tau, oracle_mod)
+
+
+def test_select_reports_rows_outside_the_domain():
+    """Rows of masses are normalised to one; a row scaled by 1e4 (its integer units would leave 64 bits) is reported
+    through the device error word instead of being cut with undefined arithmetic."""
+    shape = L.make_shape(1, 1023, 1024, 128, 128, 128, "bf16")
+    rows, nk = 8, 8
+    rng = np.random.default_rng(14)
+    mm = _masses(rng, rows, nk, "exp")
+    mm[3] *= 1e4
+    dev = torch.from_numpy(mm.ravel()).cuda()
+    indptr = torch.empty(rows + 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(rows * nk, dtype=torch.int32, device="cuda")
+    order = torch.empty(rows, dtype=torch.int32, device="cuda")
+    ws = torch.empty(L.losa_select_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    L.losa_select(shape, dev, 0.99, indptr, idx, order, ws)
+    assert L.losa_get_device_error() == -5
+    assert L.losa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("H,nb,k", [(1, 1, 1), (2, 31, 4), (4, 256, 12), (1, 929, 40), (2, 64, 64), (2, 64, 100),
+                                    (1, 929, 100), (1, 1500, 80)])
 def test_select_topk_matches_oracle(H, nb, k, oracle_mod):
     rng = np.random.default_rng(H * 7 + nb)
     m = _masses(rng, H * nb, nb, "peaked" if nb > 4 else "ties")
