@@ -32,8 +32,8 @@ constexpr uint32_t kDnQ = 0;                       // Q tile, 32 KB
 constexpr uint32_t kDnK = 32768;                   // K tile of 256 keys, 64 KB: [d-half][256 rows][128 B]
 constexpr uint32_t kDnV = 98304;                   // V tiles, 2 x 64 KB, same layout; buffer 0 doubles as mass partials
 constexpr uint32_t kDnBar = 98304 + 2 * 65536;     // barriers, TMEM slot
-constexpr uint32_t kDnXchg = kDnBar + 256;         // [2 item parity][2 groups][128] fp32 partial row sums
-constexpr uint32_t kDnSmem = kDnXchg + 2 * 2 * 128 * 4;  // 231680 bytes: needs a 1024-aligned dynamic base
+constexpr uint32_t kDnXchg = kDnBar + 256;         // [2 groups][128] (exact, rounded) fp32 partial row sums
+constexpr uint32_t kDnSmem = kDnXchg + 2 * 128 * 8;  // 231680 bytes: needs a 1024-aligned dynamic base
 
 enum : uint32_t {
     D_Q_FULL = 0, D_Q_EMPTY, D_K_FULL, D_K_EMPTY, D_V_FULL0, D_V_FULL1, D_V_EMPTY0, D_V_EMPTY1, D_S_FULL, D_S_FREE,
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t bar0 = base + kDnBar;
     auto BAR = [&](uint32_t s) { return bar0 + 8u * s; };
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kDnBar + D_COUNT * 8);
-    float* const xmax = reinterpret_cast<float*>(base_ptr + kDnXchg);           // [2 item parity][2 group][128]
+    float2* const xsum = reinterpret_cast<float2*>(base_ptr + kDnXchg);         // [2 groups][128]
     float* const part = reinterpret_cast<float*>(base_ptr + kDnV);              // [4 row groups][1024 blocks]
 
     const int warp = threadIdx.x >> 5;
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int h = w / a.nq, qb = w - h * a.nq;
             const int qrow = qb * kTcRows + row;
             const size_t grow = (size_t)h * a.Np + qrow;
-            float m_raw = -INFINITY, l_run = 0.0f;
+            float m_raw = -INFINITY, l_run = 0.0f, lr_run = 0.0f;  // exact and bf16-rounded row sums
             for (int t = 0; t < T; ++t) {
                 const int kvalid = a.N - (2 * t + (int)grp) * 128;  // real keys in this group's 128 columns
                 const bool full = kvalid >= 128;
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const float neg_mc = -m_raw * c;
                 // P for this group's 128 columns, from registers, held until the P unit is free.
                 uint32_t pw[64];
-                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)}, r2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
                 if (full) {
                     const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
 #pragma unroll
@@ -289,7 +289,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
                         float p0, p1;
                         if ((e & 3) == 3) {
-                            exp2_poly2_d3(xx, p0, p1);
+                            // the degree-4 form: these weights also enter the exact row sum behind lse, and through
+                            // it every block mass of the row (relative tolerance 1e-4)
+                            exp2_poly2(xx, p0, p1);
                         } else {
                             float x0, x1;
                             f2_unpack(xx, x0, x1);
@@ -298,6 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
                     }
                 } else {
 #pragma unroll
@@ -306,12 +309,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_mc)) : 0.0f;
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
                     }
                 }
                 float la, lb, lc, ld;
                 f2_unpack(l2[0], la, lb);
                 f2_unpack(l2[1], lc, ld);
                 l_run = l_run * alpha + ((la + lb) + (lc + ld));
+                f2_unpack(r2[0], la, lb);
+                f2_unpack(r2[1], lc, ld);
+                lr_run = lr_run * alpha + ((la + lb) + (lc + ld));
                 // The previous P V must be done before its P is overwritten and before O is rescaled.
                 if (t > 0) {
                     if (!(ok = wait_bounded_warp(BAR(D_PV_DONE), n_pv & 1u, lim))) break;
@@ -336,18 +343,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_arrive(BAR(D_P_FULL));
             }
             if (!ok) break;
-            // Epilogue: full row sum from both groups, O / l for this group's 64 columns, lse. The sums go through a
-            // buffer per item parity: the item after next writes this one again only after the next item's P V,
-            // which needs both groups' P, so both have read these sums by then.
+            // Epilogue: full row sums from both groups, O / l for this group's 64 columns, lse. A group writes the
+            // sums of the next item only after that item's first P V, or its mass phase, has needed both groups'
+            // arrivals after they read these (P_FULL, PART), so one buffer serves every item.
             if (!(ok = wait_bounded_warp(BAR(D_PV_DONE), n_pv & 1u, lim))) break;
             ++n_pv;
             tc_fence_after();
-            float* const xsum = xmax + (n_items & 1u) * 256u;
-            xsum[grp * 128u + row] = l_run;
+            xsum[grp * 128u + row] = make_float2(l_run, lr_run);
             mbar_arrive(BAR(D_SUM_X));
             if (!(ok = wait_bounded_warp(BAR(D_SUM_X), n_items & 1u, lim))) break;
-            const float l_all = l_run + xsum[(1u - grp) * 128u + row];
-            const float inv_l = 1.0f / l_all;
+            const float2 other = xsum[(1u - grp) * 128u + row];
+            const float l_all = l_run + other.x;
+            const float inv_l = 1.0f / (lr_run + other.y);
             const float lse2 = m_raw * c + lg2_approx(l_all);
             uint4* dst = reinterpret_cast<uint4*>(a.o + grow * kTcDim + grp * 64u);
 #pragma unroll

@@ -28,6 +28,10 @@ __global__ void __launch_bounds__(128) attn_f32_fwd_kernel(const F32Args a) {
     float* ks = sm_f32;
     float* vs = sm_f32 + (size_t)a.C * D;
     const int item = a.order ? a.order[blockIdx.x] : (int)blockIdx.x;
+    if (item < 0 || item >= a.H * a.nq) {  // not a permutation of the items: report it and skip the entry
+        if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrBadData);
+        return;
+    }
     const int h = item / a.nq, i = item % a.nq;
     const int r = threadIdx.x;
     const int qi = i * a.R + r;

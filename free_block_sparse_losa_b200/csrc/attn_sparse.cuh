@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         // completed, where an immediate epilogue would sit waiting for it.
         bool pend = false, sum_guard = false;  // sum_guard: the next P store waits for the last sum exchange's reads
         size_t pd_grow = 0;
-        float pd_m = 0.0f, pd_l = 0.0f;
+        float pd_m = 0.0f, pd_l = 0.0f, pd_lr = 0.0f;
         uint32_t pd_nl = 0;
         auto epilogue = [&]() -> bool {
             const uint32_t bl = pd_nl & 1u;
@@ -414,16 +414,18 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             // SUM_R, which both groups pass once they have read the other's sum.
             const uint32_t tsum = tP + bl * 64u + lane_off;
             tmem_st1(tsum + grp * 32u, __float_as_uint(pd_l));
+            tmem_st1(tsum + grp * 32u + 1u, __float_as_uint(pd_lr));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(S_SUM_X));
             if (!wait_bounded_warp(BAR(S_SUM_X), n_epi & 1u, lim)) return false;
             tc_fence_after();
             const float l_all = pd_l + __uint_as_float(tmem_ld1_wait(tsum + (grp ^ 1u) * 32u));
+            const float lr_all = pd_lr + __uint_as_float(tmem_ld1_wait(tsum + (grp ^ 1u) * 32u + 1u));
             tc_fence_before();
             mbar_arrive(BAR(S_SUM_R));
             sum_guard = true;
-            const float inv_l = 1.0f / l_all;
+            const float inv_l = 1.0f / lr_all;
             uint32_t ov[2][32];
             tmem_ld32(tO + grp * 64u + lane_off, ov[0]);
             tmem_ld32(tO + grp * 64u + lane_off + 32u, ov[1]);
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         for (int r = 0; ok && (ok = next_item(r, it, 1)) && !it.end; ++r) {
             if (it.count <= 0) continue;
             const size_t grow = (size_t)it.h * a.Np + it.qb * kTcRows + row;
-            float m_raw = -INFINITY, l_run = 0.0f;
+            float m_raw = -INFINITY, l_run = 0.0f, lr_run = 0.0f;  // exact and bf16-rounded row sums
             uint32_t kvn = it.kv4;
             for (int t = 0; t < it.tiles; ++t, ++n) {
                 const uint32_t kv4 = kvn;  // real keys per 32-column quarter of this tile
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 if (need) m_raw = (tmax == -INFINITY) ? (t == 0 ? 0.0f : m_raw) : tmax;
                 const float neg_mc = -m_raw * c;
                 uint32_t pw[32];
-                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)}, r2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
                 if (full) {
                     // one pair in four on the FMA pipe (packed degree-3 polynomial), the rest on the exp unit
                     const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
@@ -536,6 +538,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                         }
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
                     }
                 } else {
 #pragma unroll
@@ -544,12 +547,16 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                         const float p1 = (s[2 * e + 1] != -INFINITY) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_mc)) : 0.0f;
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
                     }
                 }
                 float la, lb, lc, ld;
                 f2_unpack(l2[0], la, lb);
                 f2_unpack(l2[1], lc, ld);
                 l_run = l_run * alpha + ((la + lb) + (lc + ld));
+                f2_unpack(r2[0], la, lb);
+                f2_unpack(r2[1], lc, ld);
+                lr_run = lr_run * alpha + ((la + lb) + (lc + ld));
                 // O holds the sum up to tile n - 1 once that tile's P V has completed; this group rescales its 64
                 // columns before this tile's P V may add to them.
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
@@ -588,6 +595,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             pd_grow = grow;
             pd_m = m_raw;
             pd_l = l_run;
+            pd_lr = lr_run;
             pd_nl = n - 1;
         }
         if (ok && pend) epilogue();

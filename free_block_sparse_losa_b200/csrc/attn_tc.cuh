@@ -61,6 +61,12 @@ __device__ __forceinline__ bool item_of_round(const TcArgs& a, int round, ItemIn
     const long long w = (long long)round * G + ((round & 1) ? (G - 1 - b) : b);
     if (w >= a.n_items) return false;
     it.id = a.order ? a.order[w] : (int)w;
+    if (it.id < 0 || it.id >= a.n_items) {  // not a permutation of the items: report it and skip the entry
+        atomicOr(&g_device_error, kDevErrBadData);
+        it.id = 0;
+        it.h = it.qb = it.begin = it.count = it.tiles = 0;
+        return true;
+    }
     it.h = it.id / a.nq;
     it.qb = it.id - it.h * a.nq;
     if (a.indptr) {
@@ -121,6 +127,14 @@ __device__ __forceinline__ void exp2_poly2_d3(uint64_t xx, float& r0, float& r1)
     f2_unpack(t, t0, t1);
     r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
     r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// The two fp32 values a bf16 pair from pack_bf16x2 holds (low half first), exactly, as a packed fp32 pair. The
+// attention kernels add them up per row: O is divided by the sum of the weights P V was given (the bf16-rounded P),
+// which makes O a convex combination of V rows again, so the rounding of a dominant weight cancels; the exact fp32
+// sum gives the log-sum-exp.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+    return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]^T: the A operand (P) is read from tensor memory.

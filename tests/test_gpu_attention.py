@@ -185,6 +185,41 @@ def test_sparse_reports_bad_csr():
     assert L.losa_get_device_error() == 0
 
 
+@pytest.mark.parametrize("name", ["bf16-2x(4x16x16)", "f32-tiny"])
+def test_sparse_reports_bad_work_order(name):
+    """A work-order entry outside [0, H*nq) is reported through the device error word and its slot is skipped: the
+    entry is checked before it is used, so nothing outside the inputs is read or written. Every other item is still
+    computed."""
+    cfg = SMALL[name]
+    layer = make_layer(cfg)
+    q, k, v = device_inputs(layer)
+    buf = LayerBuffers.for_config(cfg)
+    scale = scale_of(cfg)
+    buf.profile(q, k, v, scale)
+    buf.select(0.99)
+    ref = torch.empty_like(buf.o)
+    buf.sparse(q, k, v, scale, out=ref)
+    assert L.losa_get_device_error() == 0
+    good = buf.order.clone()
+    bad = good.clone()
+    bad[1] = buf.rows + 5
+    bad[2] = -1
+    buf.order.copy_(bad)
+    got = torch.zeros_like(buf.o)
+    buf.sparse(q, k, v, scale, out=got)
+    assert L.losa_get_device_error() == -5
+    assert L.losa_get_device_error() == 0
+    skipped = {int(good[1]), int(good[2])}
+    n = cfg.n_tokens
+    for it in range(buf.rows):
+        if it in skipped:
+            continue
+        h, i = divmod(it, buf.nq)
+        r0, r1 = i * cfg.block, min((i + 1) * cfg.block, n)
+        assert torch.equal(got[h, r0:r1], ref[h, r0:r1]), it
+    buf.order.copy_(good)
+
+
 def test_bounded_wait_selftest():
     """A wait on a barrier nothing completes runs out after its limit and reports LOSA_ERR_TIMEOUT; the
     context stays usable."""

@@ -107,10 +107,11 @@ def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
                 n_pv += T - 1
             yield ("wait", "PV_DONE", n_pv)
             n_pv += 1
-            yield ("put", f"XS{it & 1}h{g}", ("sum", it))
+            yield ("put", f"XSh{g}", ("sum", it))  # one exchange buffer for every item
             yield ("arrive", "SUM_X")
             yield ("wait", "SUM_X", it)
-            yield ("get", f"XS{it & 1}h{g ^ 1}", ("sum", it))
+            yield ("read", "pad")  # the read of the other group's sums may come well after the wait
+            yield ("get", f"XSh{g ^ 1}", ("sum", it))
             yield ("read", "O")
             yield ("arrive", "O_FREE")
             if with_mass:
