@@ -46,3 +46,61 @@ def test_frozen_pattern_reused_on_drifted_inputs(oracle_mod):
         gl, _ = item_rows(cfg, items, lse.cpu().numpy())
         check_output(got[valid], ref_o[valid], f"loop layer {li}")
         check_lse(gl[valid], ref_l[valid], f"loop layer {li}")
+
+
+def test_construction_at_step_three_and_cross_step_recall(oracle_mod):
+    """The LoSA page's schedule (Methodology Summary): dense steps 0, 1, 2, the pattern built at the dense step t0 = 3,
+    frozen afterwards; and its measurement of cross-step stability (Motivation Summary, "Near-lossless patterns are
+    stable across denoising"): the recall of the frozen pattern under a later step's exact masses. At construction
+    every row keeps at least tau of its own mass; at step 6 the recall the benchmark reports (from the GPU's masses)
+    equals the oracle's recall fed the same masses and lists, and agrees with the oracle's recall under its own fp64
+    masses on sampled rows; the sparse output at step 6 matches the oracle over the frozen lists."""
+    require_gpu()
+    import bench
+
+    cfg = CONFIGS["loop"]
+    layers = [make_layer(cfg, li) for li in range(2)]
+    drift = Drift(cfg, layers, seed=cfg.seed)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    tau, t0, t_probe = 0.99, 3, 6
+    bufs = [LayerBuffers.for_config(cfg) for _ in layers]
+    probe = LayerBuffers.for_config(cfg)
+    frozen = []
+    for step in range(t_probe + 1):
+        if step > 0:
+            drift.advance()
+        for li, b in enumerate(bufs):
+            q, k, v = drift.tokens(li)
+            if step < t0:
+                L.losa_dense_profile(b.shape, q, k, v, scale, b.o, b.lse, None)
+            elif step == t0:
+                b.profile(q, k, v, scale)
+                b.select(tau)
+                gi, gk, _ = b.csr_host()
+                m = b.mass.cpu().numpy().reshape(b.rows, b.nk).astype(np.float64)
+                # by construction: every row keeps >= tau of its own (GPU) mass, up to fp32 rounding of the masses
+                for r in range(b.rows):
+                    assert oracle_mod.recall(m[r:r + 1], gi[r:r + 2] - gi[r], gk[gi[r]:gi[r + 1]]) >= tau - 1e-5
+                frozen.append((gi, gk))
+            else:
+                b.sparse(q, k, v, scale)
+    assert L.losa_get_device_error() == 0
+    items = sample_items(cfg, 16, seed=5)
+    for li, b in enumerate(bufs):
+        gi, gk = frozen[li]
+        q, k, v = drift.tokens(li)
+        probe.profile(q, k, v, scale)
+        m = probe.mass.cpu().numpy().reshape(probe.rows, probe.nk).astype(np.float64)
+        r_bench = bench.pattern_recall(m, gi, gk)
+        r_oracle = oracle_mod.recall(m, gi, gk)
+        assert abs(r_bench - r_oracle) <= 1e-10 * r_oracle, (r_bench, r_oracle)
+        assert 0.0 < r_oracle <= 1.0 + 1e-6
+        qf, kf, vf = (x.float().cpu().numpy() for x in (q, k, v))
+        om = oracle_mod.mass(qf, kf, cfg.n_tokens, cfg.block, cfg.block, scale, items)
+        r_exact = oracle_mod.recall(om, gi, gk, rows=items)
+        r_gpu_rows = oracle_mod.recall(m[items], gi, gk, rows=items)
+        assert abs(r_exact - r_gpu_rows) <= 1e-4, (r_exact, r_gpu_rows)
+        ref_o, ref_l = oracle_mod.sparse(qf, kf, vf, cfg.n_tokens, cfg.block, cfg.block, scale, gi, gk, items)
+        got, valid = item_rows(cfg, items, b.o.float().cpu().numpy())
+        check_output(got[valid], ref_o[valid], f"step {t_probe} layer {li}")
+    assert L.losa_get_device_error() == 0
