@@ -147,11 +147,14 @@ losa_status losa_select_noalloc(const losa_shape* shape, const float* mass, doub
  *                   its last entry must not exceed the length of kv_block_idx: the library cannot check the
  *                   latter (it is not told that length), and a violation is undefined behaviour.
  *   order         : [H*nq] permutation of item ids giving the work order (longest list first for balance),
- *                   or NULL for ascending item order. Its entries are not checked on the device: an entry outside
- *                   [0, H*nq) is undefined behaviour (losa_select always writes a valid permutation).
+ *                   or NULL for ascending item order. An entry outside [0, H*nq) is reported and its slot skipped
+ *                   before the entry is used (losa_select always writes a valid permutation).
  *   o             : [H][Np][d] output; lse: [H][Np] fp32 output or NULL.
- * An out-of-range block index or an empty row sets the device error word (LOSA_ERR_DEVICE_FAULT); the
- * affected rows are left unspecified.
+ *   indptr, kv_block_idx and order are int32 arrays and must be 4-byte aligned (else LOSA_ERR_INVALID_ARG).
+ * An out-of-range block index, an empty row, a decreasing indptr or a bad work-order entry sets the device error
+ * word (LOSA_ERR_DEVICE_FAULT); the affected rows are left unspecified, every other row is computed.
+ * O is the restricted softmax times V with the weights rounded to bf16 for the tensor core and divided by their own
+ * sum (so O is a convex combination of the listed V rows); lse uses the exact fp32 sum.
  */
 losa_status losa_sparse_attn(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
                              const int32_t* indptr, const int32_t* kv_block_idx, const int32_t* order, void* o,
