@@ -33,7 +33,7 @@ if ROOT not in sys.path:
 from losa_synth import CONFIGS, make_layer, sample_items  # noqa: E402
 
 METRIC = "sparse-attn ms/call & dense-equiv TFLOP/s at tau=0.99; profile+select ms"
-KERNELS_PER_STEP = {"dense_profile": 1, "select": 4, "sparse_attn": 1}
+KERNELS_PER_STEP = {"dense_profile": 1, "select": 5, "sparse_attn": 1}
 
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}

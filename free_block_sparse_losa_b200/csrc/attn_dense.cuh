@@ -20,6 +20,8 @@
 //   Mass phase (same item, Q still in shared memory, lse exact in registers): S is recomputed for every 256-key tile
 //   and each warpgroup sums 2^(s*c - lse2) over its 128 columns per key block; per-warp partials go to the idle V
 //   buffer and are flushed to M every 1024 blocks.
+// Registers: the producer / MMA warpgroup drops to 56 per thread and the softmax warpgroups rise to 224 (setmaxnreg), so
+// the softmax's 128 S values, 64 P words and sums stay in registers.
 // Every wait is bounded in time (LOSA_ERR_TIMEOUT in the device error word, then a clean exit).
 #pragma once
 #include <cstdint>
@@ -86,122 +88,130 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int mass_tiles = WITH_MASS ? T : 0;
     const int G = gridDim.x;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------- TMA producer: Q and K (whole warp)
-        // Every 16 KB box of a tile is issued by its own lane (lane 0 posts the expected bytes first): one thread's
-        // TMA loads are served one after another at about 30 bytes per clock, too slow for 64 KB per tile.
-        const uint64_t pol_q = l2_policy_evict_first();
-        const uint64_t pol_kv = l2_policy_evict_last();
-        const uint32_t dh = lane >> 1, rh = lane & 1u;  // box of lane < 4: column half dh, row half rh
-        uint32_t nq = 0, nk_ld = 0;
-        bool ok = true;
-        for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
-            const int h = w / a.nq, qb = w - h * a.nq;
-            if (!(ok = wait_bounded_warp(BAR(D_Q_EMPTY), (nq & 1u) ^ 1u, lim))) break;
-            const int32_t qrow = h * a.Np + qb * kTcRows;
-            if (lane == 0) mbar_arrive_expect_tx(BAR(D_Q_FULL), kTileBytes);
-            __syncwarp();
-            if (lane < 2) tma_load_2d_hint(base + kDnQ + lane * kBoxBytes, &tmQ, 64 * (int)lane, qrow, BAR(D_Q_FULL), pol_q);
-            ++nq;
-            for (int t = 0; t < T + mass_tiles; ++t) {
-                const int32_t krow = h * a.Np + (t < T ? t : t - T) * 256;  // rows past the head are masked
-                if (!(ok = wait_bounded_warp(BAR(D_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
-                if (lane == 0) mbar_arrive_expect_tx(BAR(D_K_FULL), 2 * kTileBytes);
-                __syncwarp();
-                if (lane < 4)
-                    tma_load_2d_hint(base + kDnK + dh * 32768u + rh * 16384u, &tmK, 64 * (int)dh, krow + 128 * (int)rh,
-                                     BAR(D_K_FULL), pol_kv);
-                ++nk_ld;
-            }
-        }
-        if (nq) wait_bounded(BAR(D_Q_FULL), (nq - 1) & 1u, kDrainLimitNs);
-        if (nk_ld) wait_bounded(BAR(D_K_FULL), (nk_ld - 1) & 1u, kDrainLimitNs);
-        __syncwarp();
-    } else if (warp == 2) {
-        // ------------------------------------------------------------------- TMA producer: V (whole warp)
-        const uint64_t pol_kv = l2_policy_evict_last();
-        const uint32_t dh = lane >> 1, rh = lane & 1u;
-        uint32_t nv_ld = 0, n_it = 0;
-        bool ok = true;
-        for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
-            const int h = w / a.nq;
-            for (int t = 0; t < T; ++t) {
-                const int32_t krow = h * a.Np + t * 256;
-                const uint32_t vb = nv_ld & 1u;
-                if (!(ok = wait_bounded_warp(BAR(D_V_EMPTY0 + vb), ((nv_ld >> 1) & 1u) ^ 1u, lim))) break;
-                if (lane == 0) mbar_arrive_expect_tx(BAR(D_V_FULL0 + vb), 2 * kTileBytes);
-                __syncwarp();
-                if (lane < 4)
-                    tma_load_2d_hint(base + kDnV + vb * 65536u + dh * 32768u + rh * 16384u, &tmV, 64 * (int)dh,
-                                     krow + 128 * (int)rh, BAR(D_V_FULL0 + vb), pol_kv);
-                ++nv_ld;
-            }
-            // The mass phase reuses V buffer 0 for partial sums: before loading the next item's V, wait until the
-            // softmax has flushed this item's last chunk. MASS_DONE completes once per item, so its phase cannot be
-            // confused with a later one: the next item's needs this warp's next V loads.
-            if (WITH_MASS && ok && !(ok = wait_bounded_warp(BAR(D_MASS_DONE), n_it & 1u, lim))) break;
-            ++n_it;
-        }
-        for (uint32_t vb = 0; vb < 2; ++vb) {
-            const uint32_t n = (nv_ld + 1u - vb) >> 1;
-            if (n) wait_bounded(BAR(D_V_FULL0 + vb), (n - 1) & 1u, kDrainLimitNs);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdQK = idesc_bf16_f32(128, 256, false, false);
-            constexpr uint32_t kIdPV = idesc_bf16_f32(128, 128, false, true);
-            uint32_t nq = 0, n_qk = 0, nk_use = 0, n_pv = 0, n_items = 0;
+    // Registers: the producer / MMA warpgroup needs few, the softmax warpgroups many. Each warpgroup reaches one
+    // setmaxnreg; the split uses exactly the 384 x 168 registers the block is launched with (128 x 56 + 256 x 224).
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        if (warp == 0) {
+            // ------------------------------------------------------------- TMA producer: Q and K (whole warp)
+            // Every 16 KB box of a tile is issued by its own lane (lane 0 posts the expected bytes first): one thread's
+            // TMA loads are served one after another at about 30 bytes per clock, too slow for 64 KB per tile.
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            const uint32_t dh = lane >> 1, rh = lane & 1u;  // box of lane < 4: column half dh, row half rh
+            uint32_t nq = 0, nk_ld = 0;
             bool ok = true;
-            auto issue_pv = [&](int t) -> bool {
-                const uint32_t vb = n_pv & 1u;
-                if (!wait_bounded(BAR(D_P_FULL), n_pv & 1u, lim)) return false;
-                if (!wait_bounded(BAR(D_V_FULL0 + vb), (n_pv >> 1) & 1u, lim)) return false;
-                if (t == 0 && !wait_bounded(BAR(D_O_FREE), (n_items & 1u) ^ 1u, lim)) return false;
-                tc_fence_after();
-                const uint32_t vbase = base + kDnV + vb * 65536u;
-#pragma unroll
-                for (uint32_t h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-                    for (uint32_t kk = 0; kk < 8; ++kk)
-                        tc_mma_ts(tO, tP + h2 * 64u + kk * 8u, smem_desc(vbase + h2 * 16384u + kk * 2048u, 32768, 1024),
-                                  kIdPV, (t == 0 && h2 == 0 && kk == 0) ? 0u : 1u);
-                tc_commit(BAR(D_V_EMPTY0 + vb));
-                tc_commit(BAR(D_PV_DONE));
-                ++n_pv;
-                return true;
-            };
             for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
-                if (!(ok = wait_bounded(BAR(D_Q_FULL), nq & 1u, lim))) break;
+                const int h = w / a.nq, qb = w - h * a.nq;
+                if (!(ok = wait_bounded_warp(BAR(D_Q_EMPTY), (nq & 1u) ^ 1u, lim))) break;
+                const int32_t qrow = h * a.Np + qb * kTcRows;
+                if (lane == 0) mbar_arrive_expect_tx(BAR(D_Q_FULL), kTileBytes);
+                __syncwarp();
+                if (lane < 2) tma_load_2d_hint(base + kDnQ + lane * kBoxBytes, &tmQ, 64 * (int)lane, qrow, BAR(D_Q_FULL), pol_q);
                 ++nq;
                 for (int t = 0; t < T + mass_tiles; ++t) {
-                    if (!(ok = wait_bounded(BAR(D_K_FULL), nk_use & 1u, lim))) break;
-                    if (n_qk > 0 && !(ok = wait_bounded(BAR(D_S_FREE), (n_qk - 1) & 1u, lim))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (uint32_t kk = 0; kk < 8; ++kk) {
-                        const uint32_t qo = (kk >> 2) * kBoxBytes + (kk & 3u) * 32u;
-                        const uint32_t ko = (kk >> 2) * 32768u + (kk & 3u) * 32u;
-                        tc_mma_ss(tS, smem_desc(base + kDnQ + qo, 16, 1024), smem_desc(base + kDnK + ko, 16, 1024), kIdQK,
-                                  kk ? 1u : 0u);
-                    }
-                    tc_commit(BAR(D_S_FULL));
-                    tc_commit(BAR(D_K_EMPTY));
-                    ++nk_use;
-                    ++n_qk;
-                    if (t == T + mass_tiles - 1) tc_commit(BAR(D_Q_EMPTY));
-                    // P V of the previous forward tile goes behind this QK^T in the tensor pipe.
-                    if (t >= 1 && t <= T && !(ok = issue_pv(t - 1))) break;
+                    const int32_t krow = h * a.Np + (t < T ? t : t - T) * 256;  // rows past the head are masked
+                    if (!(ok = wait_bounded_warp(BAR(D_K_EMPTY), (nk_ld & 1u) ^ 1u, lim))) break;
+                    if (lane == 0) mbar_arrive_expect_tx(BAR(D_K_FULL), 2 * kTileBytes);
+                    __syncwarp();
+                    if (lane < 4)
+                        tma_load_2d_hint(base + kDnK + dh * 32768u + rh * 16384u, &tmK, 64 * (int)dh, krow + 128 * (int)rh,
+                                         BAR(D_K_FULL), pol_kv);
+                    ++nk_ld;
                 }
-                if (ok && mass_tiles == 0 && !(ok = issue_pv(T - 1))) break;
-                ++n_items;
             }
-            tc_commit(BAR(D_MMA_DONE));
-            wait_bounded(BAR(D_MMA_DONE), 0, kDrainLimitNs);
+            if (nq) wait_bounded(BAR(D_Q_FULL), (nq - 1) & 1u, kDrainLimitNs);
+            if (nk_ld) wait_bounded(BAR(D_K_FULL), (nk_ld - 1) & 1u, kDrainLimitNs);
+            __syncwarp();
+        } else if (warp == 2) {
+            // ------------------------------------------------------------------- TMA producer: V (whole warp)
+            const uint64_t pol_kv = l2_policy_evict_last();
+            const uint32_t dh = lane >> 1, rh = lane & 1u;
+            uint32_t nv_ld = 0, n_it = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
+                const int h = w / a.nq;
+                for (int t = 0; t < T; ++t) {
+                    const int32_t krow = h * a.Np + t * 256;
+                    const uint32_t vb = nv_ld & 1u;
+                    if (!(ok = wait_bounded_warp(BAR(D_V_EMPTY0 + vb), ((nv_ld >> 1) & 1u) ^ 1u, lim))) break;
+                    if (lane == 0) mbar_arrive_expect_tx(BAR(D_V_FULL0 + vb), 2 * kTileBytes);
+                    __syncwarp();
+                    if (lane < 4)
+                        tma_load_2d_hint(base + kDnV + vb * 65536u + dh * 32768u + rh * 16384u, &tmV, 64 * (int)dh,
+                                         krow + 128 * (int)rh, BAR(D_V_FULL0 + vb), pol_kv);
+                    ++nv_ld;
+                }
+                // The mass phase reuses V buffer 0 for partial sums: before loading the next item's V, wait until the
+                // softmax has flushed this item's last chunk. MASS_DONE completes once per item, so its phase cannot be
+                // confused with a later one: the next item's needs this warp's next V loads.
+                if (WITH_MASS && ok && !(ok = wait_bounded_warp(BAR(D_MASS_DONE), n_it & 1u, lim))) break;
+                ++n_it;
+            }
+            for (uint32_t vb = 0; vb < 2; ++vb) {
+                const uint32_t n = (nv_ld + 1u - vb) >> 1;
+                if (n) wait_bounded(BAR(D_V_FULL0 + vb), (n - 1) & 1u, kDrainLimitNs);
+            }
+            __syncwarp();
+        } else if (warp == 1) {
+            // ------------------------------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t kIdQK = idesc_bf16_f32(128, 256, false, false);
+                constexpr uint32_t kIdPV = idesc_bf16_f32(128, 128, false, true);
+                uint32_t nq = 0, n_qk = 0, nk_use = 0, n_pv = 0, n_items = 0;
+                bool ok = true;
+                auto issue_pv = [&](int t) -> bool {
+                    const uint32_t vb = n_pv & 1u;
+                    if (!wait_bounded(BAR(D_P_FULL), n_pv & 1u, lim)) return false;
+                    if (!wait_bounded(BAR(D_V_FULL0 + vb), (n_pv >> 1) & 1u, lim)) return false;
+                    if (t == 0 && !wait_bounded(BAR(D_O_FREE), (n_items & 1u) ^ 1u, lim)) return false;
+                    tc_fence_after();
+                    const uint32_t vbase = base + kDnV + vb * 65536u;
+    #pragma unroll
+                    for (uint32_t h2 = 0; h2 < 2; ++h2)
+    #pragma unroll
+                        for (uint32_t kk = 0; kk < 8; ++kk)
+                            tc_mma_ts(tO, tP + h2 * 64u + kk * 8u, smem_desc(vbase + h2 * 16384u + kk * 2048u, 32768, 1024),
+                                      kIdPV, (t == 0 && h2 == 0 && kk == 0) ? 0u : 1u);
+                    tc_commit(BAR(D_V_EMPTY0 + vb));
+                    tc_commit(BAR(D_PV_DONE));
+                    ++n_pv;
+                    return true;
+                };
+                for (int w = blockIdx.x; ok && w < a.n_items; w += G) {
+                    if (!(ok = wait_bounded(BAR(D_Q_FULL), nq & 1u, lim))) break;
+                    ++nq;
+                    for (int t = 0; t < T + mass_tiles; ++t) {
+                        if (!(ok = wait_bounded(BAR(D_K_FULL), nk_use & 1u, lim))) break;
+                        if (n_qk > 0 && !(ok = wait_bounded(BAR(D_S_FREE), (n_qk - 1) & 1u, lim))) break;
+                        tc_fence_after();
+    #pragma unroll
+                        for (uint32_t kk = 0; kk < 8; ++kk) {
+                            const uint32_t qo = (kk >> 2) * kBoxBytes + (kk & 3u) * 32u;
+                            const uint32_t ko = (kk >> 2) * 32768u + (kk & 3u) * 32u;
+                            tc_mma_ss(tS, smem_desc(base + kDnQ + qo, 16, 1024), smem_desc(base + kDnK + ko, 16, 1024), kIdQK,
+                                      kk ? 1u : 0u);
+                        }
+                        tc_commit(BAR(D_S_FULL));
+                        tc_commit(BAR(D_K_EMPTY));
+                        ++nk_use;
+                        ++n_qk;
+                        if (t == T + mass_tiles - 1) tc_commit(BAR(D_Q_EMPTY));
+                        // P V of the previous forward tile goes behind this QK^T in the tensor pipe.
+                        if (t >= 1 && t <= T && !(ok = issue_pv(t - 1))) break;
+                    }
+                    if (ok && mass_tiles == 0 && !(ok = issue_pv(T - 1))) break;
+                    ++n_items;
+                }
+                tc_commit(BAR(D_MMA_DONE));
+                wait_bounded(BAR(D_MMA_DONE), 0, kDrainLimitNs);
+            }
+            __syncwarp();
+        } else if (warp == 3) {
+            // idle: gives up its registers with the rest of its warpgroup
         }
-        __syncwarp();
-    } else if (warp >= 4) {
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
         // --------------------------------------------------------------------------- softmax warpgroups
         const uint32_t grp = (uint32_t)(warp - 4) >> 2;  // column half: keys 128 * grp .. 128 * grp + 127 of a tile
         const uint32_t wl = (uint32_t)warp & 3u;
@@ -287,17 +297,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 64; ++e) {
                         const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
-                        float p0, p1;
-                        if ((e & 3) == 3) {
-                            // the degree-4 form: these weights also enter the exact row sum behind lse, and through
-                            // it every block mass of the row (relative tolerance 1e-4)
-                            exp2_poly2(xx, p0, p1);
-                        } else {
-                            float x0, x1;
-                            f2_unpack(xx, x0, x1);
-                            p0 = ex2_approx(x0);
-                            p1 = ex2_approx(x1);
-                        }
+                        float x0, x1;
+                        f2_unpack(xx, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                         r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
@@ -405,15 +407,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 64; ++e) {
                                 const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nl2);
-                                float p0, p1;
-                                if ((e & 15) >= 9) {
-                                    exp2_poly2(xx, p0, p1);
-                                } else {
-                                    float x0, x1;
-                                    f2_unpack(xx, x0, x1);
-                                    p0 = ex2_approx(x0);
-                                    p1 = ex2_approx(x1);
-                                }
+                                float x0, x1;
+                                f2_unpack(xx, x0, x1);
+                                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                                 acc[2 * (e >> 4) + (e & 1)] = f2_add(acc[2 * (e >> 4) + (e & 1)], f2_pack(p0, p1));
                             }
                         } else {

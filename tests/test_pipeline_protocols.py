@@ -136,26 +136,29 @@ def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
 
 # -------------------------------------------------------------------------------------------------- sparse step
 
-def sparse_model(m, counts, bugs=()):
-    """attn_sparse_kernel: items read ahead through a four-entry ring, Q double-buffered, K in a 3-stage ring, V in a
-    2-stage ring whose last slot of an item takes the item's O for the TMA store, and an epilogue deferred until the
-    next item's first tile (row sums exchanged through the released P buffer)."""
+def sparse_model(m, counts, bugs=(), seed=0):
+    """attn_sparse_kernel: items read ahead through a four-entry ring, Q double-buffered in shared memory (read by every
+    Q K^T of its item, released after the last), K in a 3-stage ring, V in a 2-stage ring whose last slot of an item
+    takes the item's O for the TMA store, two S buffers and two P buffers in TMEM, a data-dependent rescale of O, and
+    an epilogue deferred until the next item's first tile (row sums exchanged through shared memory)."""
+    rng = random.Random(seed)
     RING, KST = 4, 3
     for i in range(RING):
         m.bar(f"IT_FULL{i}")
         m.bar(f"IT_EMPTY{i}", 5)  # Q/K producer, V producer, MMA issuer, two softmax warpgroups
     for i in range(2):
-        for b in ("Q_FULL", "Q_EMPTY", "V_FULL", "V_EMPTY", "PV_DONE"):
+        for b in ("Q_FULL", "Q_EMPTY", "V_FULL", "V_EMPTY", "S_FULL", "PV_DONE"):
             m.bar(f"{b}{i}")
         m.bar(f"P_FULL{i}", 2)
         m.bar(f"STAGED{i}", 2)
     for i in range(KST):
         m.bar(f"K_FULL{i}"), m.bar(f"K_EMPTY{i}")
-    for b in ("S_FULL", "MMA_DONE", "STORE_DONE"):
+    for b in ("MMA_DONE", "STORE_DONE"):
         m.bar(b)
-    for b in ("S_FREE", "SUM_R", "SUM_X", "O_FREE"):
+    for b in ("SUM_X", "O_FREE"):
         m.bar(b, 2)
     n_items = len(counts)
+    rescale = {(g, n): rng.random() < 0.4 for g in (0, 1) for n in range(sum(counts) + 2)}
 
     def next_item(r):
         yield ("wait", f"IT_FULL{r % RING}", r // RING)
@@ -240,16 +243,16 @@ def sparse_model(m, counts, bugs=()):
             qs = nq & 1
             yield ("wait", f"Q_FULL{qs}", nq >> 1)
             nq += 1
-            yield ("mma", [f"Q{qs}"], [f"TQ{items & 1}"])  # Q copied into TMEM
-            yield ("commit", f"Q_EMPTY{qs}")
             for t in range(counts[r]):
-                ks = n % KST
+                ks, b = n % KST, n & 1
                 yield ("wait", f"K_FULL{ks}", n // KST)
-                if n >= 1:
-                    yield ("wait", "S_FREE", n - 1)
-                yield ("mma", [f"TQ{items & 1}", f"K{ks}"], ["S"])
-                yield ("commit", "S_FULL")
+                yield ("mma", [f"Q{qs}", f"K{ks}"], [f"S{b}"])
+                yield ("commit", f"S_FULL{b}")
                 yield ("commit", f"K_EMPTY{ks}")
+                if t == counts[r] - 1 and "early_q_release" not in bugs:
+                    yield ("commit", f"Q_EMPTY{qs}")
+                if t == 0 and "early_q_release" in bugs:
+                    yield ("commit", f"Q_EMPTY{qs}")
                 if pend:
                     yield from issue_pv()
                 pend.update(n=n, first=t == 0, last=t == counts[r] - 1, item=items)
@@ -262,18 +265,18 @@ def sparse_model(m, counts, bugs=()):
 
     def softmax(g):
         n = n_epi = 0
-        pend, guard, nl = False, False, 0
+        pend, nl = False, 0
 
         def epilogue():
-            nonlocal n_epi, guard
+            nonlocal n_epi
             bl = nl & 1
-            yield ("wait", f"PV_DONE{bl}", nl >> 1)
-            yield ("put", f"P{bl}h{g}", ("sum", n_epi))  # partial row sum in the released P buffer
+            if "no_epilogue_pv_wait" not in bugs:
+                yield ("wait", f"PV_DONE{bl}", nl >> 1)
+            yield ("put", f"X{g}", ("sum", n_epi))  # partial row sums in shared memory
             yield ("arrive", "SUM_X")
             yield ("wait", "SUM_X", n_epi)
-            yield ("get", f"P{bl}h{g ^ 1}", ("sum", n_epi))
-            yield ("arrive", "SUM_R")
-            guard = True
+            yield ("read", "pad")  # the read of the other group's sums may come well after the wait
+            yield ("get", f"X{g ^ 1}", ("sum", n_epi))
             yield ("read", "O")
             yield ("arrive", "O_FREE")
             yield ("write", f"V{bl}")  # O staged for the TMA store
@@ -286,16 +289,13 @@ def sparse_model(m, counts, bugs=()):
                 break
             for t in range(counts[r]):
                 b = n & 1
-                yield ("wait", "S_FULL", n)
-                yield ("read", "S")
-                yield ("arrive", "S_FREE")
-                if t > 0:
-                    yield ("wait", f"PV_DONE{b ^ 1}", (n - 1) >> 1)
+                yield ("wait", f"S_FULL{b}", n >> 1)
+                yield ("read", f"S{b}")
+                if t > 0 and rescale[(g, n)]:
+                    if "no_rescale_wait" not in bugs:
+                        yield ("wait", f"PV_DONE{b ^ 1}", (n - 1) >> 1)
                     yield ("read", "O")
                     yield ("write", "O")
-                if guard and "no_sum_guard" not in bugs:
-                    yield ("wait", "SUM_R", n_epi - 1)
-                    guard = False
                 yield ("put", f"P{b}h{g}", ("p", n))
                 yield ("arrive", f"P_FULL{b}")
                 if t == 0 and pend:
@@ -331,7 +331,7 @@ def test_sparse_protocol():
     for seed in range(300):
         counts = [rng.choice([1, 1, 1, 2, 3, 5]) for _ in range(rng.randint(1, 8))]
         m = Model(seed, pipe_overlap=bool(seed & 1))
-        sparse_model(m, counts)
+        sparse_model(m, counts, seed=seed)
         m.run()
         assert not m.errors, (counts, m.errors[:3])
 
@@ -347,14 +347,14 @@ def test_dense_planted_mistakes_are_caught(bug):
     assert caught > 0
 
 
-@pytest.mark.parametrize("bug", ["no_o_free_wait", "no_sum_guard"])
+@pytest.mark.parametrize("bug", ["no_o_free_wait", "no_epilogue_pv_wait", "no_rescale_wait", "early_q_release"])
 def test_sparse_planted_mistakes_are_caught(bug):
     rng = random.Random(2)
     caught = 0
     for seed in range(120):
         counts = [rng.choice([1, 1, 2, 3]) for _ in range(rng.randint(2, 8))]
-        m = Model(seed)
-        sparse_model(m, counts, bugs=(bug,))
+        m = Model(seed, pipe_overlap=bool(seed & 1))
+        sparse_model(m, counts, bugs=(bug,), seed=seed)
         m.run()
         caught += bool(m.errors)
     assert caught > 0
