@@ -519,20 +519,13 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 uint32_t pw[32];
                 uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)}, r2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
                 if (full) {
-                    // one pair in four on the FMA pipe (packed degree-3 polynomial), the rest on the exp unit
                     const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
     #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const uint64_t xx = f2_fma(f2_pack(s[2 * e], s[2 * e + 1]), c2, nm2);
-                        float p0, p1;
-                        if ((e & 3) == 3) {
-                            exp2_poly2_d3(xx, p0, p1);
-                        } else {
-                            float x0, x1;
-                            f2_unpack(xx, x0, x1);
-                            p0 = ex2_approx(x0);
-                            p1 = ex2_approx(x1);
-                        }
+                        float x0, x1;
+                        f2_unpack(xx, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         pw[e] = pack_bf16x2(p0, p1);
                         l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                         r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));

@@ -1,5 +1,5 @@
 // Definitions shared by the tensor-core attention kernels (bf16, head_dim 128, 128-row query blocks): tile geometry,
-// the argument block, bounded mbarrier waits, work items and their key lists, the polynomial 2^x and the MMA form
+// the argument block, bounded mbarrier waits, work items and their key lists, the bf16 pair unpacking and the MMA form
 // whose A operand comes from tensor memory. The kernels are attn_dense.cuh (dense steps, with or without the block
 // masses) and attn_sparse.cuh (retained lists).
 #pragma once
@@ -79,32 +79,6 @@ __device__ __forceinline__ bool item_of_round(const TcArgs& a, int round, ItemIn
         it.tiles = a.nk;
     }
     return true;
-}
-
-// 2^x on the FMA/ALU pipes, to take part of the load off the exp unit, for weights that are rounded to bf16 (relative
-// step 2^-8) right after. Cody-Waite split x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients minimise the maximum relative
-// error on that interval (fitted by Lawson's iteratively reweighted least squares; max relative error 7.5e-5 in fp32
-// Horner form); n is added to the exponent field. Valid for x <= 126; inputs below -125 are clamped there
-// (2^-125 ~ 2.4e-38), so callers that need exact zeros (masked keys) use ex2_approx instead. Works on a pair of fp32
-// values with packed f32x2 arithmetic (the integer exponent update stays scalar).
-constexpr float kExp2D0 = 0.9999280571937561f, kExp2D1 = 0.6932609677314758f, kExp2D2 = 0.2426111251115799f,
-                kExp2D3 = 0.0551716685295105f;
-__device__ __forceinline__ void exp2_poly2_d3(uint64_t xx, float& r0, float& r1) {
-    float x0, x1;
-    f2_unpack(xx, x0, x1);
-    xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t t = f2_add(xx, f2_pack(12582912.0f, 12582912.0f));
-    const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), xx);
-    uint64_t p = f2_fma(f2_pack(kExp2D3, kExp2D3), f, f2_pack(kExp2D2, kExp2D2));
-    p = f2_fma(p, f, f2_pack(kExp2D1, kExp2D1));
-    p = f2_fma(p, f, f2_pack(kExp2D0, kExp2D0));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // The two fp32 values a bf16 pair from pack_bf16x2 holds (low half first), exactly, as a packed fp32 pair. The
