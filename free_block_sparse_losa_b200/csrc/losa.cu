@@ -263,12 +263,14 @@ size_t select_ws_bytes(const losa_shape* s) {
 losa_status launch_select_rows(const float* mass, int nk, int rows, double tau, int topk, int32_t* counts,
                                int32_t* staged, uint32_t* ticket, cudaStream_t stream) {
     const unsigned wgrid = (unsigned)((rows + 7) / 8);
+    const int sms = sm_count();
+    const unsigned sgrid = (sms > 0 && (unsigned)sms < wgrid) ? (unsigned)sms : wgrid;  // the sort kernel walks rows
 #define LOSA_ROWS_WARP(E)                                                                                        \
     do {                                                                                                         \
         select_pick_warp_kernel<E><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged, ticket); \
         const losa_status st1 = launch_status();                                                                 \
         if (st1 != LOSA_OK) return st1;                                                                          \
-        select_sort_warp_kernel<E><<<wgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);       \
+        select_sort_warp_kernel<E><<<sgrid, 256, 0, stream>>>(mass, nk, rows, tau, topk, counts, staged);       \
     } while (0)
     if (nk <= 32) LOSA_ROWS_WARP(1);
     else if (nk <= 64) LOSA_ROWS_WARP(2);

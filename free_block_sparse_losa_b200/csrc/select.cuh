@@ -11,9 +11,11 @@
 // Launches, all stream-ordered:
 //   1. select_pick_warp_kernel<E> (nk <= 1024)  one warp per row, keys in registers. At a threshold near one a row
 //        keeps a handful of blocks, so the first s positions of the sorted order are found as successive warp-wide
-//        minima of the keys above the previous pick (the pick path, up to kPickCap positions); a row whose cut lies
-//        further is left undecided (count -1) for select_sort_warp_kernel<E>, a bitonic sort of all its keys in
-//        registers. Both give the same s and kept set: the prefix runs over the same positions in the same order.
+//        minima (the pick path, up to kPickCap positions): each lane keeps its smallest unconsumed keys sorted in
+//        registers, a pick is two 32-bit warp reductions over the lanes' first entries, and a lane rescans its keys
+//        only when those are used up. A row whose cut lies further is left undecided (count -1) for
+//        select_sort_warp_kernel<E>, a bitonic sort of all its keys in registers. Both give the same s and kept
+//        set: the prefix runs over the same positions in the same order.
 //      select_pick_smem_kernel + select_rows_kernel (nk > 1024)  the pick path with the row in shared memory; rows it
 //        leaves undecided are sorted by one CTA each in shared memory.
 //      The kept blocks of each row are staged in ascending order in the workspace, with the count s.
@@ -29,8 +31,12 @@
 namespace losa {
 
 constexpr int kSelectThreads = 256;
-constexpr int kPickSlots = 2;                 // picks held per lane
+constexpr int kPickSlots = 4;                 // picks held per lane
 constexpr int kPickCap = 32 * kPickSlots;     // positions the pick path tries before falling back to the sort
+// Smallest unconsumed keys each lane keeps in registers on the pick path: two for rows in registers (where most rows
+// keep a few blocks and a rescan costs one pass over the lane's registers), four for rows in shared memory (longer
+// lists, and a rescan reads nk / 32 words of shared memory).
+constexpr int kPickCacheReg = 2, kPickCacheSmem = 4;
 constexpr int kOrderChunk = 1024;             // rows per chunk of the order kernels (one thread each)
 constexpr uint64_t kMaxRowUnits = 9007199254740992ull;          // 2^53: a row summing to 2
 
@@ -46,15 +52,6 @@ __device__ __forceinline__ uint64_t warp_incl_scan_u64(uint64_t x) {
 __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-__device__ __forceinline__ uint64_t warp_min_u64(uint64_t x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t y = __shfl_xor_sync(0xffffffffu, x, o);
-        x = y < x ? y : x;
-    }
     return x;
 }
 
@@ -154,14 +151,15 @@ __device__ __forceinline__ uint64_t sel_units(uint64_t key) {
     uint32_t bits = ~(uint32_t)(key >> 32);  // fp32 bits of a mass >= 0 (the padding key gives 0)
     bits = bits > 0x40000000u ? 0x40000000u : bits;  // min(M, 2): non-negative floats order as their bits
     const uint32_t e = bits >> 23;
-    const uint64_t m = bits & 0x7FFFFFu;
-    if (e == 0) return m ? 1ull : 0ull;
-    const int sh = (int)e - 98;
-    const uint64_t m24 = m | 0x800000u;
-    if (sh >= 0) return m24 << sh;
-    if (sh <= -25) return 1ull;  // 0 < M * 2^52 < 1/2
-    const uint32_t k = (uint32_t)(-sh);
-    return (m24 + ((1ull << k) - 1ull)) >> k;
+    const uint32_t m = bits & 0x7FFFFFu;
+    const uint64_t m24 = (uint64_t)(m | 0x800000u);
+    const int sh = (int)e - 98;  // at most 30 after the clamp
+    // Both shifts without a branch: the left one for sh >= 0; the rounded-up right one for sh < 0, where a shift by
+    // 25 or more (0 < M * 2^52 < 1/2) gives 1 because 2^23 <= m24 < 2^24.
+    const uint32_t ls = (uint32_t)(sh > 0 ? sh : 0);
+    const uint32_t rs = (uint32_t)(sh < 0 ? (sh < -25 ? 25 : -sh) : 0);
+    const uint64_t u = sh >= 0 ? (m24 << ls) : ((m24 + ((1ull << rs) - 1ull)) >> rs);
+    return e == 0 ? (m ? 1ull : 0ull) : u;
 }
 
 // Per-thread partial of a row total: capped just above the largest valid total, so that sums of partials cannot wrap
@@ -173,18 +171,39 @@ __device__ __forceinline__ uint64_t sel_target(double tau, uint64_t total) {
 }
 
 // ------------------------------------------------------------------------------------------------ pick path
-// The pick loop of one row (one warp). best: this lane's smallest key; next_above(w): this lane's smallest key above
-// w. Keys are distinct (the block index is their low word), so exactly one lane owns each pick. Returns s (> 0) when
-// the cut lies within kPickCap positions, else 0; pick t is left in lane t % 32, slot t / 32 of pk (all ones in unused
-// entries).
-template <typename NextAbove>
-__device__ __forceinline__ int pick_row(uint64_t best, uint64_t target, int want, int lane,
-                                        uint32_t (&pk)[kPickSlots], NextAbove next_above) {
+// Warp-wide minimum of 64-bit keys with two 32-bit reductions: the high words, then the low words of the lanes that
+// hold the smallest high word.
+__device__ __forceinline__ uint64_t warp_min_key(uint64_t k) {
+    const uint32_t h = (uint32_t)(k >> 32);
+    const uint32_t hm = __reduce_min_sync(0xffffffffu, h);
+    const uint32_t lm = __reduce_min_sync(0xffffffffu, h == hm ? (uint32_t)k : 0xffffffffu);
+    return ((uint64_t)hm << 32) | lm;
+}
+
+// Puts key k into the ascending list c (keeping its D smallest entries): one bubble pass.
+template <int D>
+__device__ __forceinline__ void cache_insert(uint64_t (&c)[D], uint64_t k) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+        const uint64_t lo = k < c[i] ? k : c[i];
+        k = k < c[i] ? c[i] : k;
+        c[i] = lo;
+    }
+}
+
+// The pick loop of one row (one warp). c: this lane's smallest unconsumed keys, ascending (all ones where there are
+// none), so c[0] is the lane's next candidate; refill(c, w) refills an emptied list with the lane's smallest keys
+// above w. Keys are distinct (the block index is their low word), so exactly one lane owns each pick. Returns s (> 0)
+// when the cut lies within kPickCap positions, else 0; pick t is left in lane t % 32, slot t / 32 of pk (all ones in
+// unused entries).
+template <int D, typename Refill>
+__device__ __forceinline__ int pick_row(uint64_t (&c)[D], uint64_t target, int want, int lane,
+                                        uint32_t (&pk)[kPickSlots], Refill refill) {
     uint64_t run = 0;
 #pragma unroll
     for (int p = 0; p < kPickSlots; ++p) pk[p] = 0xffffffffu;
     for (int it = 0; it < kPickCap; ++it) {
-        const uint64_t w = warp_min_u64(best);
+        const uint64_t w = warp_min_key(c[0]);
         if (w == ~0ull) return 0;  // no keys left (the cut is always reached before; kept as a guard)
         if (lane == (it & 31)) {
 #pragma unroll
@@ -192,7 +211,12 @@ __device__ __forceinline__ int pick_row(uint64_t best, uint64_t target, int want
                 if ((it >> 5) == p) pk[p] = (uint32_t)w;
         }
         run += sel_units(w);
-        if (best == w) best = next_above(w);
+        if (c[0] == w) {
+#pragma unroll
+            for (int i = 0; i + 1 < D; ++i) c[i] = c[i + 1];
+            c[D - 1] = ~0ull;
+            if (c[0] == ~0ull) refill(c, w);
+        }
         if (want ? it + 1 >= want : run >= target) return it + 1;
     }
     return 0;
@@ -200,6 +224,12 @@ __device__ __forceinline__ int pick_row(uint64_t best, uint64_t target, int want
 
 // Writes the s picked block indices of a row in ascending order.
 __device__ __forceinline__ void pick_emit(uint32_t (&pk)[kPickSlots], int s, int lane, int32_t* __restrict__ out) {
+    if (s <= 32) {  // one pick per lane (slot 0): a 32-entry sort
+        uint32_t one[1] = {pk[0]};
+        warp_bitonic_sort<1>(one, lane);
+        if (lane < s) out[lane] = (int32_t)one[0];
+        return;
+    }
     warp_bitonic_sort<kPickSlots>(pk, lane);
 #pragma unroll
     for (int p = 0; p < kPickSlots; ++p)
@@ -225,35 +255,42 @@ __global__ void __launch_bounds__(256, 2) select_pick_warp_kernel(const float* _
     const float* m = mass + (size_t)row * nk;
     uint32_t hi[E];  // high words of the keys of blocks e * 32 + lane
     bool bad = false;
-    uint64_t local = 0, best = ~0ull;
+    uint64_t local = 0, c[kPickCacheReg];
+#pragma unroll
+    for (int i = 0; i < kPickCacheReg; ++i) c[i] = ~0ull;
+    float mv[E];  // every load of the row goes out before the first use
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int j = e * 32 + lane;
-        const uint64_t key = (j < nk) ? sel_key(m[j], (uint32_t)j, bad) : ((0xFFFFFFFFull << 32) | (uint32_t)j);
+        mv[e] = (j < nk) ? __ldg(m + j) : 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = e * 32 + lane;
+        const uint64_t key = (j < nk) ? sel_key(mv[e], (uint32_t)j, bad) : ((0xFFFFFFFFull << 32) | (uint32_t)j);
         hi[e] = (uint32_t)(key >> 32);
         local += sel_units(key);
-        best = key < best ? key : best;
+        cache_insert(c, key);
     }
     const uint64_t total = warp_sum_u64(cap_units(local));
     if (topk == 0 && total > kMaxRowUnits) bad = true;
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_device_error, kDevErrBadData);
     const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
     uint32_t pk[kPickSlots];
-    const int s = (want > kPickCap) ? 0 : pick_row(best, sel_target(tau, total), want, lane, pk, [&](uint64_t w) {
-        uint64_t b = ~0ull;
+    const int s = (want > kPickCap) ? 0 : pick_row(c, sel_target(tau, total), want, lane, pk,
+                                                   [&](uint64_t (&cc)[kPickCacheReg], uint64_t w) {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
             const uint64_t key = ((uint64_t)hi[e] << 32) | (uint32_t)(e * 32 + lane);
-            b = (key > w && key < b) ? key : b;
+            cache_insert(cc, key > w ? key : ~0ull);
         }
-        return b;
     });
     if (s > 0) pick_emit(pk, s, lane, staged + (size_t)row * nk);
     if (lane == 0) counts[row] = s > 0 ? s : -1;
 }
 
-// Kernel 1b, register form: the rows kernel 1a left undecided (count -1; other warps return at once), each sorted
-// whole by one warp in registers; lane l then holds sorted positions l*E .. l*E+E-1.
+// Kernel 1b, register form: the rows kernel 1a left undecided (count -1), each sorted whole by one warp in registers;
+// lane l then holds sorted positions l*E .. l*E+E-1.
 template <int E>
 __global__ void __launch_bounds__(256) select_sort_warp_kernel(const float* __restrict__ mass, int nk, int rows,
                                                                 double tau, int topk, int32_t* __restrict__ counts,
@@ -261,69 +298,78 @@ __global__ void __launch_bounds__(256) select_sort_warp_kernel(const float* __re
     __shared__ uint32_t bitmap_all[8][32];
     const int warp = threadIdx.x >> 5;
     const int lane = (int)lane_id();
-    const int row = blockIdx.x * 8 + warp;
-    if (row >= rows || counts[row] >= 0) return;  // warp-uniform
-    const float* m = mass + (size_t)row * nk;
-    uint64_t key[E];
-    bool bad = false;  // reported by kernel 1a, which read the same row
-    uint64_t local = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int j = e * 32 + lane;
-        key[e] = (j < nk) ? sel_key(m[j], (uint32_t)j, bad) : ~0ull;
-        local += sel_units(key[e]);
-    }
-    const uint64_t target = sel_target(tau, warp_sum_u64(cap_units(local)));
-    const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
-    int32_t* out = staged + (size_t)row * nk;
-    warp_bitonic_sort<E>(key, lane);
-    uint64_t ls = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) ls += sel_units(key[e]);
-    const uint64_t incl = warp_incl_scan_u64(cap_units(ls));
-    uint64_t run = incl - cap_units(ls);
-    int below = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        run += sel_units(key[e]);
-        below += (run < target) ? 1 : 0;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
-    int s = (below + 1 < nk) ? below + 1 : nk;
-    if (want) s = want;
-    // Kept set (sorted positions < s) -> bitmap by block index -> ascending compaction.
-    uint32_t* bitmap = bitmap_all[warp];
-    for (int w = lane; w < E; w += 32) bitmap[w] = 0u;
-    __syncwarp();
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (lane * E + e < s) {
-            const uint32_t j = (uint32_t)(key[e] & 0xffffffffu);
-            atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+    // a grid of at most one CTA per SM walks the rows; decided rows cost one load of their count
+    for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+        if (counts[row] >= 0) continue;  // warp-uniform
+        const float* m = mass + (size_t)row * nk;
+        uint64_t key[E];
+        bool bad = false;  // reported by kernel 1a, which read the same row
+        uint64_t local = 0;
+        float mv[E];  // every load of the row goes out before the first use
+    #pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int j = e * 32 + lane;
+            mv[e] = (j < nk) ? __ldg(m + j) : 0.0f;
         }
-    __syncwarp();
-    // Lane l emits the kept blocks among [l*E, l*E + E) at its exclusive prefix of kept counts.
-    uint32_t myb = 0;
-    const int j0 = lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int j = j0 + e;
-        if (j < nk && ((bitmap[j >> 5] >> (j & 31)) & 1u)) myb |= 1u << e;
+    #pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int j = e * 32 + lane;
+            key[e] = (j < nk) ? sel_key(mv[e], (uint32_t)j, bad) : ~0ull;
+            local += sel_units(key[e]);
+        }
+        const uint64_t target = sel_target(tau, warp_sum_u64(cap_units(local)));
+        const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
+        int32_t* out = staged + (size_t)row * nk;
+        warp_bitonic_sort<E>(key, lane);
+        uint64_t ls = 0;
+    #pragma unroll
+        for (int e = 0; e < E; ++e) ls += sel_units(key[e]);
+        const uint64_t incl = warp_incl_scan_u64(cap_units(ls));
+        uint64_t run = incl - cap_units(ls);
+        int below = 0;
+    #pragma unroll
+        for (int e = 0; e < E; ++e) {
+            run += sel_units(key[e]);
+            below += (run < target) ? 1 : 0;
+        }
+    #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+        int s = (below + 1 < nk) ? below + 1 : nk;
+        if (want) s = want;
+        // Kept set (sorted positions < s) -> bitmap by block index -> ascending compaction.
+        uint32_t* bitmap = bitmap_all[warp];
+        for (int w = lane; w < E; w += 32) bitmap[w] = 0u;
+        __syncwarp();
+    #pragma unroll
+        for (int e = 0; e < E; ++e)
+            if (lane * E + e < s) {
+                const uint32_t j = (uint32_t)(key[e] & 0xffffffffu);
+                atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+            }
+        __syncwarp();
+        // Lane l emits the kept blocks among [l*E, l*E + E) at its exclusive prefix of kept counts.
+        uint32_t myb = 0;
+        const int j0 = lane * E;
+    #pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int j = j0 + e;
+            if (j < nk && ((bitmap[j >> 5] >> (j & 31)) & 1u)) myb |= 1u << e;
+        }
+        const int cnt = __popc(myb);
+        int pre = cnt;
+    #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += y;
+        }
+        pre -= cnt;
+    #pragma unroll
+        for (int e = 0; e < E; ++e)
+            if ((myb >> e) & 1u) out[pre++] = j0 + e;
+        __syncwarp();
+        if (lane == 0) counts[row] = s;
+        __syncwarp();  // the bitmap is reused by the warp's next row
     }
-    const int cnt = __popc(myb);
-    int pre = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, pre, o);
-        if (lane >= o) pre += y;
-    }
-    pre -= cnt;
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if ((myb >> e) & 1u) out[pre++] = j0 + e;
-    __syncwarp();
-    if (lane == 0) counts[row] = s;
 }
 
 // Kernel 1a for nk > 1024: the pick path with the row in shared memory. W = blockDim.x / 32 warps, one row each;
@@ -342,12 +388,23 @@ __global__ void __launch_bounds__(256) select_pick_smem_kernel(const float* __re
     uint32_t* kb = pick_bits + (size_t)warp * nk;
     const float* m = mass + (size_t)row * nk;
     bool bad = false;
-    uint64_t local = 0, best = ~0ull;
-    for (int j = lane; j < nk; j += 32) {
-        const uint64_t k = sel_key(m[j], (uint32_t)j, bad);
-        kb[j] = (uint32_t)(k >> 32);
-        local += sel_units(k);
-        best = k < best ? k : best;
+    uint64_t local = 0, c[kPickCacheSmem];
+#pragma unroll
+    for (int i = 0; i < kPickCacheSmem; ++i) c[i] = ~0ull;
+    for (int j0 = lane; j0 < nk; j0 += 32 * 8) {  // eight loads in flight per lane before their first use
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = (j0 + 32 * u < nk) ? __ldg(m + j0 + 32 * u) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = j0 + 32 * u;
+            if (j < nk) {
+                const uint64_t k = sel_key(v[u], (uint32_t)j, bad);
+                kb[j] = (uint32_t)(k >> 32);
+                local += sel_units(k);
+                cache_insert(c, k);
+            }
+        }
     }
     __syncwarp();
     const uint64_t total = warp_sum_u64(cap_units(local));
@@ -355,13 +412,12 @@ __global__ void __launch_bounds__(256) select_pick_smem_kernel(const float* __re
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&g_device_error, kDevErrBadData);
     const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
     uint32_t pk[kPickSlots];
-    const int s = (want > kPickCap) ? 0 : pick_row(best, sel_target(tau, total), want, lane, pk, [&](uint64_t w) {
-        uint64_t b = ~0ull;
+    const int s = (want > kPickCap) ? 0 : pick_row(c, sel_target(tau, total), want, lane, pk,
+                                                   [&](uint64_t (&cc)[kPickCacheSmem], uint64_t w) {
         for (int j = lane; j < nk; j += 32) {
             const uint64_t k = ((uint64_t)kb[j] << 32) | (uint32_t)j;
-            b = (k > w && k < b) ? k : b;
+            cache_insert(cc, k > w ? k : ~0ull);
         }
-        return b;
     });
     if (s > 0) pick_emit(pk, s, lane, staged + (size_t)row * nk);
     if (lane == 0) counts[row] = s > 0 ? s : -1;
@@ -381,14 +437,22 @@ __global__ void __launch_bounds__(NT) select_rows_kernel(const float* __restrict
     const int row = blockIdx.x;
     if (counts[row] >= 0) return;  // the pick kernel has cut this row (and reported any bad data)
     const float* m = mass + (size_t)row * nk;
-    for (int j = threadIdx.x; j < n2; j += NT) {
-        uint64_t key = ~0ull;
-        if (j < nk) {
-            bool bad = false;  // reported by the pick kernel, which read the same row
-            key = sel_key(m[j], (uint32_t)j, bad);
-            kept[j] = 0;
+    for (int j0 = threadIdx.x; j0 < n2; j0 += NT * 4) {  // four loads in flight per thread before their first use
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = (j0 + NT * u < nk) ? __ldg(m + j0 + NT * u) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + NT * u;
+            if (j >= n2) break;
+            uint64_t key = ~0ull;
+            if (j < nk) {
+                bool bad = false;  // reported by the pick kernel, which read the same row
+                key = sel_key(v[u], (uint32_t)j, bad);
+                kept[j] = 0;
+            }
+            keys[j] = key;
         }
-        keys[j] = key;
     }
     __syncthreads();
 
