@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(256, 2) select_pick_warp_kernel(const float* _
                                                                 double tau, int topk, int32_t* __restrict__ counts,
                                                                 int32_t* __restrict__ staged,
                                                                 uint32_t* __restrict__ ticket) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
+    if (blockIdx.x == 0 && threadIdx.x == 0) ticket[0] = ticket[1] = 0u;  // the order kernels' counter and max
     const int warp = threadIdx.x >> 5;
     const int lane = (int)lane_id();
     const int row = blockIdx.x * 8 + warp;
@@ -298,77 +298,81 @@ __global__ void __launch_bounds__(256) select_sort_warp_kernel(const float* __re
     __shared__ uint32_t bitmap_all[8][32];
     const int warp = threadIdx.x >> 5;
     const int lane = (int)lane_id();
-    // a grid of at most one CTA per SM walks the rows; decided rows cost one load of their count
-    for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
-        if (counts[row] >= 0) continue;  // warp-uniform
-        const float* m = mass + (size_t)row * nk;
-        uint64_t key[E];
-        bool bad = false;  // reported by kernel 1a, which read the same row
-        uint64_t local = 0;
-        float mv[E];  // every load of the row goes out before the first use
+    // A grid of at most one CTA per SM walks the rows in chunks of 32: one coalesced load of the chunk's counts, then
+    // the undecided rows of the chunk one after another.
+    for (int base = (blockIdx.x * 8 + warp) * 32; base < rows; base += gridDim.x * 8 * 32) {
+        uint32_t todo = __ballot_sync(0xffffffffu, base + lane < rows && counts[base + lane] < 0);
+        for (; todo; todo &= todo - 1u) {
+            const int row = base + (__ffs(todo) - 1);
+            const float* m = mass + (size_t)row * nk;
+            uint64_t key[E];
+            bool bad = false;  // reported by kernel 1a, which read the same row
+            uint64_t local = 0;
+            float mv[E];  // every load of the row goes out before the first use
     #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int j = e * 32 + lane;
-            mv[e] = (j < nk) ? __ldg(m + j) : 0.0f;
-        }
-    #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int j = e * 32 + lane;
-            key[e] = (j < nk) ? sel_key(mv[e], (uint32_t)j, bad) : ~0ull;
-            local += sel_units(key[e]);
-        }
-        const uint64_t target = sel_target(tau, warp_sum_u64(cap_units(local)));
-        const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
-        int32_t* out = staged + (size_t)row * nk;
-        warp_bitonic_sort<E>(key, lane);
-        uint64_t ls = 0;
-    #pragma unroll
-        for (int e = 0; e < E; ++e) ls += sel_units(key[e]);
-        const uint64_t incl = warp_incl_scan_u64(cap_units(ls));
-        uint64_t run = incl - cap_units(ls);
-        int below = 0;
-    #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            run += sel_units(key[e]);
-            below += (run < target) ? 1 : 0;
-        }
-    #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
-        int s = (below + 1 < nk) ? below + 1 : nk;
-        if (want) s = want;
-        // Kept set (sorted positions < s) -> bitmap by block index -> ascending compaction.
-        uint32_t* bitmap = bitmap_all[warp];
-        for (int w = lane; w < E; w += 32) bitmap[w] = 0u;
-        __syncwarp();
-    #pragma unroll
-        for (int e = 0; e < E; ++e)
-            if (lane * E + e < s) {
-                const uint32_t j = (uint32_t)(key[e] & 0xffffffffu);
-                atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+            for (int e = 0; e < E; ++e) {
+                const int j = e * 32 + lane;
+                mv[e] = (j < nk) ? __ldg(m + j) : 0.0f;
             }
-        __syncwarp();
-        // Lane l emits the kept blocks among [l*E, l*E + E) at its exclusive prefix of kept counts.
-        uint32_t myb = 0;
-        const int j0 = lane * E;
     #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int j = j0 + e;
-            if (j < nk && ((bitmap[j >> 5] >> (j & 31)) & 1u)) myb |= 1u << e;
+            for (int e = 0; e < E; ++e) {
+                const int j = e * 32 + lane;
+                key[e] = (j < nk) ? sel_key(mv[e], (uint32_t)j, bad) : ~0ull;
+                local += sel_units(key[e]);
+            }
+            const uint64_t target = sel_target(tau, warp_sum_u64(cap_units(local)));
+            const int want = topk > 0 ? (topk < nk ? topk : nk) : 0;
+            int32_t* out = staged + (size_t)row * nk;
+            warp_bitonic_sort<E>(key, lane);
+            uint64_t ls = 0;
+    #pragma unroll
+            for (int e = 0; e < E; ++e) ls += sel_units(key[e]);
+            const uint64_t incl = warp_incl_scan_u64(cap_units(ls));
+            uint64_t run = incl - cap_units(ls);
+            int below = 0;
+    #pragma unroll
+            for (int e = 0; e < E; ++e) {
+                run += sel_units(key[e]);
+                below += (run < target) ? 1 : 0;
+            }
+    #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+            int s = (below + 1 < nk) ? below + 1 : nk;
+            if (want) s = want;
+            // Kept set (sorted positions < s) -> bitmap by block index -> ascending compaction.
+            uint32_t* bitmap = bitmap_all[warp];
+            for (int w = lane; w < E; w += 32) bitmap[w] = 0u;
+            __syncwarp();
+    #pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (lane * E + e < s) {
+                    const uint32_t j = (uint32_t)(key[e] & 0xffffffffu);
+                    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                }
+            __syncwarp();
+            // Lane l emits the kept blocks among [l*E, l*E + E) at its exclusive prefix of kept counts.
+            uint32_t myb = 0;
+            const int j0 = lane * E;
+    #pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = j0 + e;
+                if (j < nk && ((bitmap[j >> 5] >> (j & 31)) & 1u)) myb |= 1u << e;
+            }
+            const int cnt = __popc(myb);
+            int pre = cnt;
+    #pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, pre, o);
+                if (lane >= o) pre += y;
+            }
+            pre -= cnt;
+    #pragma unroll
+            for (int e = 0; e < E; ++e)
+                if ((myb >> e) & 1u) out[pre++] = j0 + e;
+            __syncwarp();
+            if (lane == 0) counts[row] = s;
+            __syncwarp();  // the bitmap is reused by the warp's next row
         }
-        const int cnt = __popc(myb);
-        int pre = cnt;
-    #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, pre, o);
-            if (lane >= o) pre += y;
-        }
-        pre -= cnt;
-    #pragma unroll
-        for (int e = 0; e < E; ++e)
-            if ((myb >> e) & 1u) out[pre++] = j0 + e;
-        __syncwarp();
-        if (lane == 0) counts[row] = s;
-        __syncwarp();  // the bitmap is reused by the warp's next row
     }
 }
 
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(256) select_pick_smem_kernel(const float* __re
                                                                 int32_t* __restrict__ staged,
                                                                 uint32_t* __restrict__ ticket) {
     extern __shared__ __align__(16) uint32_t pick_bits[];
-    if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
+    if (blockIdx.x == 0 && threadIdx.x == 0) ticket[0] = ticket[1] = 0u;  // the order kernels' counter and max
     const int warp = threadIdx.x >> 5;
     const int lane = (int)lane_id();
     const int row = blockIdx.x * (int)(blockDim.x >> 5) + warp;
@@ -527,6 +531,8 @@ __global__ void __launch_bounds__(kOrderChunk) select_hist_kernel(const int32_t*
         }
         atomicAdd(&hist[nk - c], 1);
     }
+    const int cmax = __reduce_max_sync(0xffffffffu, c);
+    if ((threadIdx.x & 31u) == 0 && cmax > 0) atomicMax(&ticket[1], (uint32_t)cmax);  // the longest list anywhere
     uint64_t tot;
     block_excl_scan_u64<kOrderChunk>((uint64_t)c, warp_tot, tot);  // also orders the histogram updates
     for (int b = threadIdx.x; b < nk; b += kOrderChunk) table[(size_t)b * nch + blockIdx.x] = hist[b];
@@ -539,12 +545,16 @@ __global__ void __launch_bounds__(kOrderChunk) select_hist_kernel(const int32_t*
     __threadfence();
     // The last chunk: exclusive scan of table (n = nk * nch entries) in linear order, kScanSeg entries at a time.
     // Each segment is loaded with coalesced reads into shared memory (the histogram space, free again), where every
-    // thread scans kScanPer contiguous entries; the running total carries from segment to segment.
+    // thread scans kScanPer contiguous entries; the running total carries from segment to segment. The bins of counts
+    // above the longest list are empty, so the scan starts at the bin of that count: every entry before it is zero
+    // and none is read by the order kernel.
     constexpr int kScanPer = 8, kScanSeg = kOrderChunk * kScanPer;
     __shared__ int32_t seg[kScanSeg];  // 32 KB
     const size_t n = (size_t)nk * nch;
+    const uint32_t lmax = __ldcg(&ticket[1]);
+    const size_t first = (size_t)(nk - (int)(lmax < 1u ? 1u : (lmax > (uint32_t)nk ? (uint32_t)nk : lmax))) * nch;
     uint64_t carry = 0;
-    for (size_t s0 = 0; s0 < n; s0 += kScanSeg) {
+    for (size_t s0 = first; s0 < n; s0 += kScanSeg) {
         const int cnt = (int)min((size_t)kScanSeg, n - s0);
 #pragma unroll
         for (int u = 0; u < kScanPer; ++u) {
@@ -582,7 +592,7 @@ __global__ void __launch_bounds__(kOrderChunk) select_hist_kernel(const int32_t*
     if (threadIdx.x < (unsigned)nch) chunk_off[threadIdx.x] = (int64_t)cpre;
     if (threadIdx.x == 0) {
         indptr[rows] = (int32_t)total;
-        *ticket = 0u;
+        ticket[0] = ticket[1] = 0u;
     }
 }
 
