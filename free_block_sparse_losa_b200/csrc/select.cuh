@@ -135,18 +135,17 @@ __device__ __forceinline__ void warp_bitonic_sort(T (&key)[E], int lane) {
 // masses), low word = j (ascending among equal masses). A negative, NaN or infinite mass sets bad and counts as 0;
 // -0 counts as +0. Padding keys (all ones) sort last.
 __device__ __forceinline__ uint64_t sel_key(float x, uint32_t j, bool& bad) {
-    if (!(x >= 0.0f) || isinf(x)) {
-        bad = true;
-        x = 0.0f;
-    }
-    const uint32_t bits = (x == 0.0f) ? 0u : __float_as_uint(x);
-    return ((uint64_t)(~bits) << 32) | j;
+    uint32_t bits = __float_as_uint(x);
+    bits = (bits == 0x80000000u) ? 0u : bits;  // -0 is 0
+    const bool ok = bits < 0x7F800000u;          // finite and not negative
+    bad |= !ok;
+    return ((uint64_t)(~(ok ? bits : 0u)) << 32) | j;
 }
 
 // u = ceil(min(M, 2) * 2^52) of a key's mass (0 for the padding key), in integer arithmetic on the fp32 fields:
 // M = m24 * 2^(e - 150) for a normal mass, so M * 2^52 = m24 * 2^(e - 98), a shift or a rounded-up shift; a
 // subnormal mass is below 2^-126 and gives 1. The result equals ceil(M * 2^52) taken in fp64, which is exact. Masses
-// above 2 lie outside the input domain (the row-sum check reports them); the clamp keeps every unit below 2^53 + 1.
+// above 2 lie outside the input domain (the row-sum check reports them); the clamp keeps every unit at most 2^53.
 __device__ __forceinline__ uint64_t sel_units(uint64_t key) {
     uint32_t bits = ~(uint32_t)(key >> 32);  // fp32 bits of a mass >= 0 (the padding key gives 0)
     bits = bits > 0x40000000u ? 0x40000000u : bits;  // min(M, 2): non-negative floats order as their bits
@@ -160,6 +159,17 @@ __device__ __forceinline__ uint64_t sel_units(uint64_t key) {
     const uint32_t rs = (uint32_t)(sh < 0 ? (sh < -25 ? 25 : -sh) : 0);
     const uint64_t u = sh >= 0 ? (m24 << ls) : ((m24 + ((1ull << rs) - 1ull)) >> rs);
     return e == 0 ? (m ? 1ull : 0ull) : u;
+}
+
+// The same units through the conversion unit: the scaling by 2^52 only moves the exponent (min(M, 2) * 2^52 <= 2^53,
+// and a subnormal M becomes a normal number) and the conversion rounds up, so the result is exactly the ceiling; a
+// subnormal mass gives 1 whatever the compiler's handling of subnormal operands. Fewer instructions, but the 64-bit
+// conversion has a low rate: the shared-memory pick path (latency-bound) uses this form, the register path (issue-
+// bound) the integer one.
+__device__ __forceinline__ uint64_t sel_units_cvt(uint64_t key) {
+    const uint32_t bits = ~(uint32_t)(key >> 32);
+    const uint64_t u = __float2ull_ru(fminf(__uint_as_float(bits), 2.0f) * 4503599627370496.0f);
+    return (bits - 1u < 0x7FFFFFu) ? 1ull : u;
 }
 
 // Per-thread partial of a row total: capped just above the largest valid total, so that sums of partials cannot wrap
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__(256) select_pick_smem_kernel(const float* __re
             if (j < nk) {
                 const uint64_t k = sel_key(v[u], (uint32_t)j, bad);
                 kb[j] = (uint32_t)(k >> 32);
-                local += sel_units(k);
+                local += sel_units_cvt(k);
                 cache_insert(c, k);
             }
         }
