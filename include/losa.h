@@ -98,7 +98,8 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
  * integer prefix makes the result independent of summation order, and tau = 1 keeps exactly the non-zero blocks.
  * A negative or non-finite mass sets the device error word (LOSA_ERR_DEVICE_FAULT) and is treated as zero. A row
  * summing to more than 2 sets it too, and that row's list is unspecified (units are formed from min(M_j, 2), so
- * nothing overflows and no arithmetic is undefined). Four stream-ordered launches: the per-row cut, per-chunk histograms of the list
+ * nothing overflows and no arithmetic is undefined). Five stream-ordered launches: the per-row cut (a pick pass for
+ * rows that keep up to 128 blocks, then a full sort of the rows it leaves undecided), per-chunk histograms of the list
  * lengths, indptr with the work order, and the copy of the lists into place.
  */
 losa_status losa_select(const losa_shape* shape, const float* mass, double tau, int32_t* indptr,
@@ -129,8 +130,8 @@ size_t losa_select_workspace_bytes(const losa_shape* shape);
  *   admits H * nq * nk up to about 4.1 million (a 12-head layer of 256 x 256 blocks needs 3.2 MB).
  *   The library allocates nothing in this call. Its first call on a device (and the first after a device reset, which
  *   loads the library's device code again) looks up the array's device address, which may load the library's device
- *   code onto that device, so make that first call before any stream capture. The call's first kernel clears the one
- *   counter in the array that must start at zero.
+ *   code onto that device, so make that first call before any stream capture. The call's first kernel clears the two
+ *   words in the array that must start at zero (a completion counter and the longest list length).
  *   Every call on a device shares the one array and overwrites what the previous call left there: calls whose GPU
  *   work can overlap (different streams without ordering between them) race on it and must be serialised.
  */
