@@ -75,8 +75,9 @@ def work_model(cfg, nnz):
     nq, nkb, C = Np // B, Np // cfg.kblock, cfg.kblock
     return {
         "dense_equiv_flop": 4.0 * H * N * N * d,
-        "profile_flop": 6.0 * H * N * N * d,          # Q K^T + P V forward, then Q K^T again for the masses
-        "profile_exp": 2.0 * H * N * N,
+        # Q K^T + P V of the forward; the block masses come from the forward's own weights (one pass)
+        "profile_flop": 4.0 * H * N * N * d,
+        "profile_exp": 1.0 * H * N * N,
         "sparse_flop": 4.0 * B * C * d * nnz,         # kept blocks only (R x C each)
         "sparse_exp": float(B * C * nnz),
         "select_bytes": 4.0 * H * nq * nkb + 4.0 * (nnz + 2 * H * nq + 1),  # read M, write CSR + order

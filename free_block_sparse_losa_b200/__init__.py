@@ -60,6 +60,9 @@ def load():
                                   ctypes.c_int64, ctypes.c_size_t)
     sp = ctypes.POINTER(LosaShape)
     L.losa_dense_profile.argtypes = [sp, vp, vp, vp, f32, vp, vp, vp, vp]
+    L.losa_dense_profile_ws.argtypes = [sp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
+    L.losa_dense_profile_workspace_bytes.argtypes = [sp]
+    L.losa_dense_profile_workspace_bytes.restype = sz
     L.losa_select.argtypes = [sp, vp, f64, vp, vp, i64, vp, vp, sz, vp]
     L.losa_select_noalloc.argtypes = [sp, vp, f64, vp, vp, i64, vp, vp]
     L.losa_select_topk.argtypes = [sp, vp, i32, vp, vp, i64, vp, vp, sz, vp]
@@ -73,7 +76,8 @@ def load():
     L.losa_status_string.argtypes = [i32]
     L.losa_status_string.restype = ctypes.c_char_p
     L.losa_version.restype = ctypes.c_int
-    for name in ("losa_dense_profile", "losa_select", "losa_select_noalloc", "losa_select_topk", "losa_sparse_attn",
+    for name in ("losa_dense_profile", "losa_dense_profile_ws", "losa_select", "losa_select_noalloc", "losa_select_topk",
+                 "losa_sparse_attn",
                  "losa_get_device_error",
                  "losa_selftest_wait_timeout"):
         getattr(L, name).restype = i32
@@ -141,6 +145,34 @@ def losa_dense_profile(shape, q, k, v, scale, o, lse=None, mass=None, stream=Non
                                    (mass, "mass", "float32", H * nq * nk))
     st = load().losa_dense_profile(ctypes.byref(shape), pq, pk, pv, float(scale), po, pl, pm, _stream(stream))
     return _check(st, "losa_dense_profile", raise_on_error)
+
+
+def losa_dense_profile_workspace_bytes(shape) -> int:
+    return int(load().losa_dense_profile_workspace_bytes(ctypes.byref(shape)))
+
+
+def losa_dense_profile_ws(shape, q, k, v, scale, o, lse, mass, workspace, ws_bytes=None, stream=None,
+                          raise_on_error=True):
+    """losa_dense_profile with the masses taken in the forward pass (needs a workspace of
+    losa_dense_profile_workspace_bytes(shape) bytes)."""
+    H, Np, d, nq, nk = _dims(shape)
+    tdt = _token_dtype(shape)
+    if isinstance(workspace, int):
+        if ws_bytes is None:
+            raise ValueError("workspace: a raw pointer needs ws_bytes")
+        wsb = int(ws_bytes)
+    else:
+        have = workspace.numel() * workspace.element_size()
+        wsb = have if ws_bytes is None else int(ws_bytes)
+        if have < wsb:
+            raise ValueError(f"workspace: holds {have} bytes, ws_bytes says {wsb}")
+    pq, pk, pv, po, pl, pm, pw = _ptrs((q, "q", tdt, H * Np * d), (k, "k", tdt, H * Np * d),
+                                       (v, "v", tdt, H * Np * d), (o, "o", tdt, H * Np * d),
+                                       (lse, "lse", "float32", H * Np), (mass, "mass", "float32", H * nq * nk),
+                                       (workspace, "workspace", None, None))
+    st = load().losa_dense_profile_ws(ctypes.byref(shape), pq, pk, pv, float(scale), po, pl, pm, pw, wsb,
+                                      _stream(stream))
+    return _check(st, "losa_dense_profile_ws", raise_on_error)
 
 
 def losa_select_workspace_bytes(shape) -> int:

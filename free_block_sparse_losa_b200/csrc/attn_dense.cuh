@@ -35,14 +35,19 @@ constexpr uint32_t kDnK = 32768;                   // K tile of 256 keys, 64 KB:
 constexpr uint32_t kDnV = 98304;                   // V tiles, 2 x 64 KB, same layout; buffer 0 doubles as mass partials
 constexpr uint32_t kDnBar = 98304 + 2 * 65536;     // barriers, TMEM slot
 constexpr uint32_t kDnXchg = kDnBar + 256;         // [2 groups][128] (exact, rounded) fp32 partial row sums
-constexpr uint32_t kDnSmem = kDnXchg + 2 * 128 * 8;  // 231680 bytes: needs a 1024-aligned dynamic base
+constexpr uint32_t kDnFsc = kDnXchg + 2 * 128 * 8;   // [128] fp32 row factors of the one-pass mass reduction
+constexpr uint32_t kDnSmem = kDnFsc + 128 * 4;       // 232192 bytes: needs a 1024-aligned dynamic base
+static_assert(kDnSmem <= 232448, "shared memory");
+// One-pass masses: a row's stored block sums stay relative to its anchor max m0 while the running max stays within
+// 2^kAnchorSpan of it (so no stored sum can overflow); past that the row re-anchors and rescales what it stored.
+constexpr float kAnchorSpan = 60.0f;
 
 enum : uint32_t {
     D_Q_FULL = 0, D_Q_EMPTY, D_K_FULL, D_K_EMPTY, D_V_FULL0, D_V_FULL1, D_V_EMPTY0, D_V_EMPTY1, D_S_FULL, D_S_FREE,
     D_P_FULL, D_PV_DONE, D_O_FREE, D_SUM_X, D_PART, D_PART2, D_MASS_DONE, D_MMA_DONE, D_COUNT
 };
 
-template <bool WITH_MASS, int SUB>
+template <bool WITH_MASS, int SUB, bool ONE_PASS = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_dense_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -58,6 +63,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kDnBar + D_COUNT * 8);
     float2* const xsum = reinterpret_cast<float2*>(base_ptr + kDnXchg);         // [2 groups][128]
     float* const part = reinterpret_cast<float*>(base_ptr + kDnV);              // [4 row groups][1024 blocks]
+    float* const fsc = reinterpret_cast<float*>(base_ptr + kDnFsc);             // [128] one-pass row factors
 
     const int warp = threadIdx.x >> 5;
     const uint32_t lane = lane_id();
@@ -85,7 +91,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tS = tmem, tO = tmem + 256u, tP = tmem + 384u;
     const unsigned long long lim = a.wait_limit_ns;
     const int T = (a.nk + 1) / 2;  // 256-key tiles per head
-    const int mass_tiles = WITH_MASS ? T : 0;
+    const int mass_tiles = (WITH_MASS && !ONE_PASS) ? T : 0;  // the two-pass form recomputes every tile
     const int G = gridDim.x;
 
     // Registers: the producer / MMA warpgroup needs few, the softmax warpgroups many. Each warpgroup reaches one
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // The mass phase reuses V buffer 0 for partial sums: before loading the next item's V, wait until the
                 // softmax has flushed this item's last chunk. MASS_DONE completes once per item, so its phase cannot be
                 // confused with a later one: the next item's needs this warp's next V loads.
-                if (WITH_MASS && ok && !(ok = wait_bounded_warp(BAR(D_MASS_DONE), n_it & 1u, lim))) break;
+                if (WITH_MASS && !ONE_PASS && ok && !(ok = wait_bounded_warp(BAR(D_MASS_DONE), n_it & 1u, lim))) break;
                 ++n_it;
             }
             for (uint32_t vb = 0; vb < 2; ++vb) {
@@ -226,6 +232,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int qrow = qb * kTcRows + row;
             const size_t grow = (size_t)h * a.Np + qrow;
             float m_raw = -INFINITY, l_run = 0.0f, lr_run = 0.0f;  // exact and bf16-rounded row sums
+            // one-pass masses: this row's anchor max and the factor from the current reference max to it
+            float m0 = 0.0f, fac = 1.0f;
+            float* const pslot = ONE_PASS ? a.mass_part + (size_t)blockIdx.x * a.nkb * kTcRows : nullptr;
             for (int t = 0; t < T; ++t) {
                 const int kvalid = a.N - (2 * t + (int)grp) * 128;  // real keys in this group's 128 columns
                 const bool full = kvalid >= 128;
@@ -289,9 +298,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const float alpha = (t > 0 && need) ? ex2_approx((m_raw - tmax) * c) : 1.0f;
                 if (need) m_raw = tmax;
                 const float neg_mc = -m_raw * c;
-                // P for this group's 128 columns, from registers, held until the P unit is free.
+                // P for this group's 128 columns, from registers, held until the P unit is free. The one-pass mass
+                // with 32-key blocks keeps the exact sums per 32 columns (lq), the others per pair parity (l2).
+                constexpr bool kQuarters = ONE_PASS && SUB > 1;
                 uint32_t pw[64];
                 uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)}, r2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                uint64_t lq[kQuarters ? 8 : 1];
+#pragma unroll
+                for (int i = 0; i < (kQuarters ? 8 : 1); ++i) lq[i] = f2_pack(0.f, 0.f);
                 if (full) {
                     const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(neg_mc, neg_mc);
 #pragma unroll
@@ -301,7 +315,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         f2_unpack(xx, x0, x1);
                         const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         pw[e] = pack_bf16x2(p0, p1);
-                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        if constexpr (kQuarters)
+                            lq[2 * (e >> 4) + (e & 1)] = f2_add(lq[2 * (e >> 4) + (e & 1)], f2_pack(p0, p1));
+                        else
+                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                         r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
                     }
                 } else {
@@ -310,17 +327,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const float p0 = (2 * e < kvalid) ? ex2_approx(fmaf(s[2 * e], c, neg_mc)) : 0.0f;
                         const float p1 = (2 * e + 1 < kvalid) ? ex2_approx(fmaf(s[2 * e + 1], c, neg_mc)) : 0.0f;
                         pw[e] = pack_bf16x2(p0, p1);
-                        l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
+                        if constexpr (kQuarters)
+                            lq[2 * (e >> 4) + (e & 1)] = f2_add(lq[2 * (e >> 4) + (e & 1)], f2_pack(p0, p1));
+                        else
+                            l2[e & 1] = f2_add(l2[e & 1], f2_pack(p0, p1));
                         r2[e & 1] = f2_add(r2[e & 1], bf16x2_to_f2(pw[e]));
+                    }
+                }
+                float qs[kQuarters ? 4 : 1];  // exact sums of the 32-column quarters
+                if constexpr (kQuarters) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float x0, x1, x2, x3;
+                        f2_unpack(lq[2 * g], x0, x1);
+                        f2_unpack(lq[2 * g + 1], x2, x3);
+                        qs[g] = (x0 + x1) + (x2 + x3);
                     }
                 }
                 float la, lb, lc, ld;
                 f2_unpack(l2[0], la, lb);
                 f2_unpack(l2[1], lc, ld);
-                l_run = l_run * alpha + ((la + lb) + (lc + ld));
+                float tsum;  // exact sum of this tile's 128 columns
+                if constexpr (kQuarters)
+                    tsum = (qs[0] + qs[1]) + (qs[2] + qs[3]);
+                else
+                    tsum = (la + lb) + (lc + ld);
+                l_run = l_run * alpha + tsum;
                 f2_unpack(r2[0], la, lb);
                 f2_unpack(r2[1], lc, ld);
                 lr_run = lr_run * alpha + ((la + lb) + (lc + ld));
+                if constexpr (ONE_PASS) {
+                    // This tile's block sums of 2^(s c - m0 c), for the reduction at the item's end. The reference
+                    // max only grows; past 2^kAnchorSpan above the anchor the row re-anchors first (rare).
+                    if (t == 0) {
+                        m0 = m_raw;
+                        fac = 1.0f;
+                    } else if (need) {
+                        if ((m_raw - m0) * c > kAnchorSpan) {
+                            const float r = ex2_approx((m0 - m_raw) * c);
+                            for (int tt = 0; tt < t; ++tt)
+                                for (int g = 0; g < SUB; ++g) {
+                                    const int j = (2 * tt + (int)grp) * SUB + g;
+                                    if (j < a.nkb) pslot[(size_t)j * kTcRows + row] *= r;
+                                }
+                            m0 = m_raw;
+                            fac = 1.0f;
+                        } else {
+                            fac = ex2_approx((m_raw - m0) * c);
+                        }
+                    }
+                    if constexpr (kQuarters) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int j = (2 * t + (int)grp) * SUB + g;
+                            if (j < a.nkb) pslot[(size_t)j * kTcRows + row] = qs[g] * fac;
+                        }
+                    } else {
+                        const int j = 2 * t + (int)grp;
+                        if (j < a.nkb) pslot[(size_t)j * kTcRows + row] = tsum * fac;
+                    }
+                }
                 // The previous P V must be done before its P is overwritten and before O is rescaled.
                 if (t > 0) {
                     if (!(ok = wait_bounded_warp(BAR(D_PV_DONE), n_pv & 1u, lim))) break;
@@ -378,7 +444,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_arrive(BAR(D_O_FREE));
             if (a.lse && grp == 0) a.lse[grow] = lse2 * 0.6931471805599453f;
 
-            if (WITH_MASS) {
+            if constexpr (ONE_PASS) {
+                // M(i, j) = sum over the block's rows of (stored sum) * 2^(m0 c - m c) / l, divided by its real rows.
+                // Every row's sums were stored before the row-sum exchange above; the factors go through shared
+                // memory; the next item overwrites both only after every warp has passed PART2.
+                if (grp == 0) fsc[row] = (qrow < a.N) ? ex2_approx((m0 - m_raw) * c) / l_all : 0.0f;
+                mbar_arrive(BAR(D_PART));
+                if (!(ok = wait_bounded_warp(BAR(D_PART), n_items & 1u, lim))) break;
+                const float inv_rows = 1.0f / (float)min(kTcRows, a.N - qb * kTcRows);
+                float* mrow = a.mass + (size_t)w * a.nkb;
+                const float4 f4 = reinterpret_cast<const float4*>(fsc)[lane];
+                for (int j = warp - 4; j < a.nkb; j += 8) {
+                    const float4 v4 = reinterpret_cast<const float4*>(pslot + (size_t)j * kTcRows)[lane];
+                    float sum = (v4.x * f4.x + v4.y * f4.y) + (v4.z * f4.z + v4.w * f4.w);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                    if (lane == 0) mrow[j] = sum * inv_rows;
+                }
+                mbar_arrive(BAR(D_PART2));
+                if (!(ok = wait_bounded_warp(BAR(D_PART2), n_items & 1u, lim))) break;
+            }
+
+            if (WITH_MASS && !ONE_PASS) {
                 // Mass phase: 2^(s*c - lse2) summed per key block of this group's columns, for real rows and keys.
                 const bool qvalid = qrow < a.N;
                 const float neg_lse2 = qvalid ? -lse2 : 0.0f;

@@ -27,6 +27,7 @@ struct TcArgs {
     __nv_bfloat16* o;
     float* lse;                    // may be null
     float* mass;                   // [H*nq][nk], WITH_MASS only
+    float* mass_part;              // one-pass masses: per-CTA scratch of [nkb][128] fp32 partial sums (else null)
     unsigned long long wait_limit_ns;
 };
 

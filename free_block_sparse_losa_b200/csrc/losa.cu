@@ -109,13 +109,13 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint32_t bo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool M, int SUB>
+template <bool M, int SUB, bool ONE_PASS = false>
 losa_status launch_dense_kernel(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const TcArgs& a, cudaStream_t stream) {
-    if (cudaFuncSetAttribute(attn_dense_kernel<M, SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDnSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_dense_kernel<M, SUB, ONE_PASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kDnSmem) != cudaSuccess)
         return LOSA_ERR_CUDA;
-    attn_dense_kernel<M, SUB><<<grid, kTcThreads, kDnSmem, stream>>>(tq, tk, tv, a);
+    attn_dense_kernel<M, SUB, ONE_PASS><<<grid, kTcThreads, kDnSmem, stream>>>(tq, tk, tv, a);
     return launch_status();
 }
 
@@ -134,7 +134,7 @@ losa_status launch_sparse_kernel(int grid, const CUtensorMap& tq, const CUtensor
 // without a list, the sparse-step kernel with one.
 losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const void* k, const void* v, float scale,
                       const int32_t* indptr, const int32_t* kv_idx, const int32_t* order, void* o, float* lse,
-                      float* mass, cudaStream_t stream) {
+                      float* mass, cudaStream_t stream, float* mass_part = nullptr) {
     const uint64_t rows = (uint64_t)s->heads * s->n_padded;
     const bool c32 = s->block_k == 32;
     CUtensorMap tq, tk, tv, tk32, tv32;
@@ -160,12 +160,16 @@ losa_status launch_tc(const losa_shape* s, bool with_mass, const void* q, const 
     a.o = static_cast<__nv_bfloat16*>(o);
     a.lse = lse;
     a.mass = mass;
+    a.mass_part = mass_part;
     a.wait_limit_ns = g_wait_limit_ns;
     const int sms = sm_count();
     if (sms <= 0) return LOSA_ERR_CUDA;
     if (!indptr) {
         // dense step: one item per CTA at a time, 256-key tiles
         const int dgrid = a.n_items < sms ? a.n_items : sms;
+        if (with_mass && mass_part)  // one pass: block sums from the forward, reduced per item (dgrid scratch slots)
+            return c32 ? launch_dense_kernel<true, 4, true>(dgrid, tq, tk, tv, a, stream)
+                       : launch_dense_kernel<true, 1, true>(dgrid, tq, tk, tv, a, stream);
         if (with_mass)
             return c32 ? launch_dense_kernel<true, 4>(dgrid, tq, tk, tv, a, stream)
                        : launch_dense_kernel<true, 1>(dgrid, tq, tk, tv, a, stream);
@@ -387,6 +391,30 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
         return launch_f32<128>(shape, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, mass, stream);
     }
     return LOSA_ERR_UNSUPPORTED;
+}
+
+size_t losa_dense_profile_workspace_bytes(const losa_shape* shape) {
+    if (check_shape(shape) != LOSA_OK || !tc_shape(shape)) return 0;
+    const int sms = sm_count();
+    if (sms <= 0) return 0;
+    return (size_t)sms * (size_t)(shape->n_padded / shape->block_k) * kTcRows * sizeof(float);
+}
+
+losa_status losa_dense_profile_ws(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                  void* o, float* lse, float* mass, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    if (!mass || !tc_shape(shape)) return losa_dense_profile(shape, q, k, v, scale, o, lse, mass, stream);
+    losa_status st = check_shape(shape);
+    if (st != LOSA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(mass) ||
+        !aligned16(workspace))
+        return LOSA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return LOSA_ERR_INVALID_ARG;
+    const size_t need = losa_dense_profile_workspace_bytes(shape);
+    if (need == 0) return LOSA_ERR_CUDA;
+    if (ws_bytes < need) return LOSA_ERR_CAPACITY;
+    return launch_tc(shape, true, q, k, v, scale, nullptr, nullptr, nullptr, o, lse, mass, stream,
+                     static_cast<float*>(workspace));
 }
 
 size_t losa_select_workspace_bytes(const losa_shape* shape) {

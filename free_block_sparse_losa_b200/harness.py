@@ -8,8 +8,8 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from . import (DTYPE_BF16, DTYPE_F32, losa_dense_profile, losa_select, losa_select_topk, losa_select_workspace_bytes,
-               losa_sparse_attn, make_shape)
+from . import (DTYPE_BF16, DTYPE_F32, losa_dense_profile, losa_dense_profile_workspace_bytes, losa_dense_profile_ws,
+               losa_select, losa_select_topk, losa_select_workspace_bytes, losa_sparse_attn, make_shape)
 
 
 def host_tokens_to_device(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
@@ -52,15 +52,23 @@ class LayerBuffers:
         self.order = torch.empty(self.rows, dtype=torch.int32, device=dev)
         ws = losa_select_workspace_bytes(self.shape)
         self.workspace = torch.empty((ws + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+        pws = losa_dense_profile_workspace_bytes(self.shape)  # 0 on the fp32 path
+        self.profile_workspace = torch.empty(max(16, (pws + 15) // 16 * 16), dtype=torch.uint8, device=dev)
 
     @classmethod
     def for_config(cls, cfg, device="cuda"):
         return cls(cfg.heads, cfg.n_tokens, cfg.n_padded, cfg.head_dim, cfg.block, cfg.dtype, device,
                    getattr(cfg, "block_k", 0))
 
-    def profile(self, q, k, v, scale, with_mass=True, stream=None):
-        losa_dense_profile(self.shape, q, k, v, scale, self.o, self.lse, self.mass if with_mass else None,
-                           stream=stream)
+    def profile(self, q, k, v, scale, with_mass=True, stream=None, one_pass=True):
+        """The dense step; with_mass adds the block masses, in the forward pass (one_pass, the default) or in a
+        second pass that needs no workspace."""
+        if with_mass and one_pass:
+            losa_dense_profile_ws(self.shape, q, k, v, scale, self.o, self.lse, self.mass, self.profile_workspace,
+                                  stream=stream)
+        else:
+            losa_dense_profile(self.shape, q, k, v, scale, self.o, self.lse, self.mass if with_mass else None,
+                               stream=stream)
 
     def select(self, tau, mass=None, stream=None):
         losa_select(self.shape, self.mass if mass is None else mass, tau, self.indptr, self.kv_idx, self.order,

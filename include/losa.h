@@ -79,6 +79,25 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
                                void* o, float* lse, float* mass, cudaStream_t stream);
 
 /*
+ * The dense profiling step with the masses taken in the same pass as the forward, at the cost of a scratch buffer:
+ * the same arguments and results as losa_dense_profile (same definitions; the masses agree with it and with the exact
+ * values within the same 1e-4 relative bound, not bit for bit: the sums run in another order).
+ *   workspace : device scratch of at least losa_dense_profile_workspace_bytes(shape) bytes (16-byte aligned),
+ *               contents on entry irrelevant; ws_bytes is its size, else LOSA_ERR_CAPACITY before any launch.
+ * The forward pass already forms every weight 2^(s c - m c) against the row's running max m; it keeps, per row and
+ * key block, the exact sum of those weights (brought to one anchor max per row) in the scratch, and each item's
+ * masses are reduced from them once the row's final log-sum-exp is known: one pass over the keys instead of two.
+ * With mass == NULL, or on the fp32 path, the call is losa_dense_profile and the workspace is not touched.
+ */
+losa_status losa_dense_profile_ws(const losa_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                  void* o, float* lse, float* mass, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+/* Scratch bytes losa_dense_profile_ws needs on the current device (SM count x nk x 128 fp32); 0 for an invalid
+ * shape or the fp32 path. */
+size_t losa_dense_profile_workspace_bytes(const losa_shape* shape);
+
+/*
  * Mass-threshold selection (LoSA page, Methodology Summary, "One-time pattern construction": sort the key
  * blocks of one (head, query block) by decreasing mass and keep the shortest prefix whose mass reaches
  * theta times the block's total).

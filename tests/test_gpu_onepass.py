@@ -1,0 +1,93 @@
+"""The block masses taken in the forward pass (losa_dense_profile_ws; LoSA page, Motivation Summary, M(i, j) as the
+sum of A over a query block and a key block) against the two-pass call and the oracle: on small layers at C = 128
+and C = 32, on a layer whose later keys raise each row's max far above its first tile's (the row's anchor moves and
+its stored sums are rescaled), and the call's refusals."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import free_block_sparse_losa_b200 as L
+from free_block_sparse_losa_b200.harness import LayerBuffers
+from losa_synth import make_layer
+from tests.gpu_util import check_lse, check_mass, check_output, device_inputs, item_rows, require_gpu, scale_of
+from tests.test_gpu_attention import SMALL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _both_ways(cfg, layer, oracle):
+    """Runs the two-pass and the one-pass profile on the same inputs; checks the one-pass masses, O and lse against
+    the oracle, and O against the two-pass call bit for bit (the forward is the same code)."""
+    q, k, v = device_inputs(layer)
+    buf = LayerBuffers.for_config(cfg)
+    scale = scale_of(cfg)
+    buf.profile(q, k, v, scale, one_pass=False)
+    m2, o2, l2 = buf.mass.cpu().numpy().copy(), buf.o.clone(), buf.lse.clone()
+    buf.profile(q, k, v, scale)
+    torch.cuda.synchronize()
+    assert L.losa_get_device_error() == 0
+    assert torch.equal(buf.o.view(torch.int16), o2.view(torch.int16))
+    assert float((buf.lse - l2).abs().max()) <= 1e-5
+    items = np.arange(buf.rows, dtype=np.int32)
+    qf, kf, vf = layer.all_f32("q"), layer.all_f32("k"), layer.all_f32("v")
+    ref = oracle.mass(qf, kf, cfg.n_tokens, cfg.block, cfg.kblock, scale, items)
+    m1 = buf.mass.cpu().numpy().reshape(buf.rows, buf.nk)
+    check_mass(m1, ref, f"{cfg.name} one-pass")
+    check_mass(m2.reshape(buf.rows, buf.nk), ref, f"{cfg.name} two-pass")
+    np.testing.assert_allclose(m1.sum(axis=1), 1.0, atol=1e-3)
+    od, ld = oracle.dense(qf, kf, vf, cfg.n_tokens, cfg.block, scale, items)
+    go, valid = item_rows(cfg, items, buf.o.float().cpu().numpy())
+    gl, _ = item_rows(cfg, items, buf.lse.cpu().numpy())
+    check_output(go[valid], od[valid], f"{cfg.name} dense O")
+    check_lse(gl[valid], ld[valid], f"{cfg.name} dense lse")
+
+
+@pytest.mark.parametrize("name", ["bf16-3x(5x13x31)-ragged", "bf16-C32-3x(5x13x31)-ragged",
+                                  "bf16-1x(1x1x77)-one-block"])
+def test_one_pass_masses(name, oracle_mod):
+    cfg = SMALL[name]
+    _both_ways(cfg, make_layer(cfg), oracle_mod)
+
+
+def _scale_keys(layer, t0, t1, log2_factor):
+    """The keys of tokens t0 .. t1 - 1 of every head times 2^log2_factor, exactly (the bf16 exponent field)."""
+    k = layer.k.astype(np.int32)
+    seg = k[:, t0:t1]
+    k[:, t0:t1] = np.where((seg & 0x7FFF) != 0, seg + (log2_factor << 7), seg)
+    return dataclasses.replace(layer, k=k.astype(np.uint16))
+
+
+@pytest.mark.parametrize("name", ["bf16-3x(5x13x31)-ragged", "bf16-C32-3x(5x13x31)-ragged"])
+def test_one_pass_masses_when_the_row_max_grows_far(name, oracle_mod):
+    cfg = SMALL[name]
+    layer = make_layer(cfg)
+    n = cfg.n_tokens
+    # a middle tile 4x (the reference max moves within the anchor span), the last tile 16x (far past it)
+    layer = _scale_keys(layer, 512, 768, 2)
+    layer = _scale_keys(layer, (n - 1) // 256 * 256, n, 4)
+    _both_ways(cfg, layer, oracle_mod)
+
+
+def test_one_pass_refusals():
+    cfg = SMALL["bf16-2x(4x16x16)"]
+    q, k, v = device_inputs(make_layer(cfg))
+    buf = LayerBuffers.for_config(cfg)
+    need = L.losa_dense_profile_workspace_bytes(buf.shape)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert need == sms * buf.nk * 128 * 4
+    scale = scale_of(cfg)
+    st = L.losa_dense_profile_ws(buf.shape, q, k, v, scale, buf.o, buf.lse, buf.mass, buf.profile_workspace,
+                                 ws_bytes=need - 1, raise_on_error=False)
+    assert st == -3  # LOSA_ERR_CAPACITY
+    st = L.losa_dense_profile_ws(buf.shape, q, k, v, scale, buf.o, buf.lse, buf.mass,
+                                 buf.profile_workspace.data_ptr() + 4, ws_bytes=need, raise_on_error=False)
+    assert st == -1  # LOSA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert L.losa_get_device_error() == 0
