@@ -22,9 +22,16 @@ def _gpu():
     require_gpu()
 
 
-def _both_ways(cfg, layer, oracle):
-    """Runs the two-pass and the one-pass profile on the same inputs; checks the one-pass masses, O and lse against
-    the oracle, and O against the two-pass call bit for bit (the forward is the same code)."""
+def _check_mass_rtol(gpu_rows, ref_rows, rtol, what):
+    err = np.abs(gpu_rows.astype(np.float64) - ref_rows)
+    bad = err > rtol * ref_rows + 1e-30
+    assert not bad.any(), f"{what}: {int(bad.sum())} entries beyond {rtol} relative, first at {np.argwhere(bad)[0]}"
+
+
+def _both_ways(cfg, layer, oracle, mass_rtol=None):
+    """Runs the two-pass and the one-pass profile on the same inputs; checks both calls' masses, and the one-pass
+    call's O and lse, against the oracle, and O against the two-pass call bit for bit (the forward is the same
+    code). mass_rtol replaces the 1e-4 mass tolerance where the inputs make fp32 logits too coarse for it."""
     q, k, v = device_inputs(layer)
     buf = LayerBuffers.for_config(cfg)
     scale = scale_of(cfg)
@@ -39,8 +46,12 @@ def _both_ways(cfg, layer, oracle):
     qf, kf, vf = layer.all_f32("q"), layer.all_f32("k"), layer.all_f32("v")
     ref = oracle.mass(qf, kf, cfg.n_tokens, cfg.block, cfg.kblock, scale, items)
     m1 = buf.mass.cpu().numpy().reshape(buf.rows, buf.nk)
-    check_mass(m1, ref, f"{cfg.name} one-pass")
-    check_mass(m2.reshape(buf.rows, buf.nk), ref, f"{cfg.name} two-pass")
+    if mass_rtol is None:
+        check_mass(m1, ref, f"{cfg.name} one-pass")
+        check_mass(m2.reshape(buf.rows, buf.nk), ref, f"{cfg.name} two-pass")
+    else:
+        _check_mass_rtol(m1, ref, mass_rtol, f"{cfg.name} one-pass")
+        _check_mass_rtol(m2.reshape(buf.rows, buf.nk), ref, mass_rtol, f"{cfg.name} two-pass")
     np.testing.assert_allclose(m1.sum(axis=1), 1.0, atol=1e-3)
     od, ld = oracle.dense(qf, kf, vf, cfg.n_tokens, cfg.block, scale, items)
     go, valid = item_rows(cfg, items, buf.o.float().cpu().numpy())
@@ -69,10 +80,13 @@ def test_one_pass_masses_when_the_row_max_grows_far(name, oracle_mod):
     cfg = SMALL[name]
     layer = make_layer(cfg)
     n = cfg.n_tokens
-    # a middle tile 4x (the reference max moves within the anchor span), the last tile 16x (far past it)
+    # a middle tile 4x (the reference max moves within the anchor span), the last tile 16x (far past it). The last
+    # tile's logits reach about 1000, where one fp32 ulp of the tensor core's accumulation is about 1e-4 of the
+    # logit scale times log2(e): both calls then agree with the exact masses to a few 1e-5, at times just above
+    # 1e-4, so this case checks the anchor logic at 5e-4 (a wrong anchor factor would be off by 2^60).
     layer = _scale_keys(layer, 512, 768, 2)
     layer = _scale_keys(layer, (n - 1) // 256 * 256, n, 4)
-    _both_ways(cfg, layer, oracle_mod)
+    _both_ways(cfg, layer, oracle_mod, mass_rtol=5e-4)
 
 
 def test_one_pass_refusals():
