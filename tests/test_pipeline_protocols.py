@@ -19,13 +19,17 @@ from tests.pipeline_model import Model
 
 def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
     """attn_dense_kernel: one query block per item, T key tiles (single-buffered K, double-buffered V); with the mass
-    phase, T more Q K^T tiles whose block sums are reduced through V buffer 0."""
+    phase (with_mass True), T more Q K^T tiles whose block sums are reduced through V buffer 0; with one-pass masses
+    (with_mass "one_pass"), each forward tile's block sums stored to the workspace (W{g}) and reduced by both groups
+    after the row sums are known, with the row factors in shared memory (F) between the PART and PART2 barriers."""
+    one_pass = with_mass == "one_pass"
+    two_pass = bool(with_mass) and not one_pass
     for b in ("Q_FULL", "Q_EMPTY", "K_FULL", "K_EMPTY", "S_FULL", "PV_DONE", "MMA_DONE",
               "V_FULL0", "V_FULL1", "V_EMPTY0", "V_EMPTY1"):
         m.bar(b)
     for b in ("S_FREE", "P_FULL", "O_FREE", "SUM_X", "PART", "PART2", "MASS_DONE"):
         m.bar(b, 2)  # both softmax warpgroups
-    mass_tiles = T if with_mass else 0
+    mass_tiles = T if two_pass else 0
 
     def qk_producer():
         nq = nk = 0
@@ -49,7 +53,7 @@ def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
                 yield ("expect", f"V_FULL{vb}", 1)
                 yield ("tma", f"V_FULL{vb}", 1, f"V{vb}")
                 nv += 1
-            if with_mass:
+            if two_pass:
                 yield ("wait", "MASS_DONE", it)
 
     def mma():
@@ -102,6 +106,8 @@ def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
                     yield ("read", "O")  # rescale of this group's half of O
                     yield ("write", "O")
                 yield ("put", f"Ph{g}", ("p", it, t))
+                if one_pass:
+                    yield ("put", f"W{g}", ("sums", it, t))  # this tile's block sums of its rows
                 yield ("arrive", "P_FULL")
             if "no_pv_wait_before_p" in bugs:
                 n_pv += T - 1
@@ -114,7 +120,19 @@ def dense_model(m, n_items, T, with_mass, chunk_tiles, bugs=()):
             yield ("get", f"XSh{g ^ 1}", ("sum", it))
             yield ("read", "O")
             yield ("arrive", "O_FREE")
-            if with_mass:
+            if one_pass:
+                if g == 0:
+                    yield ("put", "F", ("factors", it))
+                yield ("arrive", "PART")
+                if "no_part_wait" not in bugs:
+                    yield ("wait", "PART", it)
+                yield ("get", "F", ("factors", it))
+                yield ("get", "W0", ("sums", it, T - 1))  # the reduction reads both groups' stored sums
+                yield ("get", "W1", ("sums", it, T - 1))
+                yield ("arrive", "PART2")
+                if "no_part2_wait" not in bugs:
+                    yield ("wait", "PART2", it)
+            if two_pass:
                 for t0 in range(0, T, chunk_tiles):
                     for _ in range(t0, min(T, t0 + chunk_tiles)):
                         yield ("wait", "S_FULL", n_s)
@@ -313,7 +331,7 @@ def sparse_model(m, counts, bugs=(), seed=0):
 # -------------------------------------------------------------------------------------------------------- tests
 
 def _dense_cases():
-    return [(n_items, T, mass, chunk) for n_items in (1, 3) for T in (1, 2, 5) for mass in (False, True)
+    return [(n_items, T, mass, chunk) for n_items in (1, 3) for T in (1, 2, 5) for mass in (False, True, "one_pass")
             for chunk in (1, 2)]
 
 
@@ -336,12 +354,13 @@ def test_sparse_protocol():
         assert not m.errors, (counts, m.errors[:3])
 
 
-@pytest.mark.parametrize("bug", ["no_s_free_wait", "no_pv_wait_before_p"])
-def test_dense_planted_mistakes_are_caught(bug):
+@pytest.mark.parametrize("bug,mode", [("no_s_free_wait", True), ("no_pv_wait_before_p", True),
+                                      ("no_part_wait", "one_pass"), ("no_part2_wait", "one_pass")])
+def test_dense_planted_mistakes_are_caught(bug, mode):
     caught = 0
     for seed in range(40):
         m = Model(seed)
-        dense_model(m, 3, 3, True, 2, bugs=(bug,))
+        dense_model(m, 3, 3, mode, 2, bugs=(bug,))
         m.run()
         caught += bool(m.errors)
     assert caught > 0
