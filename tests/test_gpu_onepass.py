@@ -41,7 +41,10 @@ def _both_ways(cfg, layer, oracle, mass_rtol=None):
     torch.cuda.synchronize()
     assert L.losa_get_device_error() == 0
     assert torch.equal(buf.o.view(torch.int16), o2.view(torch.int16))
-    assert float((buf.lse - l2).abs().max()) <= 1e-5
+    # lse = m + ln l: with C = 32 the one-pass call sums each row's weights in four quarter accumulators, so l may
+    # differ from the two-pass call's by a few fp32 ulps, and lse by a few ulps of its own size (about 900 on the
+    # scaled-key layer, where one ulp is 6e-5)
+    assert bool(((buf.lse - l2).abs() <= 1e-5 + 4 * 2.0 ** -23 * l2.abs()).all())
     items = np.arange(buf.rows, dtype=np.int32)
     qf, kf, vf = layer.all_f32("q"), layer.all_f32("k"), layer.all_f32("v")
     ref = oracle.mass(qf, kf, cfg.n_tokens, cfg.block, cfg.kblock, scale, items)
