@@ -28,10 +28,11 @@ def _check_mass_rtol(gpu_rows, ref_rows, rtol, what):
     assert not bad.any(), f"{what}: {int(bad.sum())} entries beyond {rtol} relative, first at {np.argwhere(bad)[0]}"
 
 
-def _both_ways(cfg, layer, oracle, mass_rtol=None):
+def _both_ways(cfg, layer, oracle, mass_rtol=None, lse_rtol=0.0):
     """Runs the two-pass and the one-pass profile on the same inputs; checks both calls' masses, and the one-pass
     call's O and lse, against the oracle, and O against the two-pass call bit for bit (the forward is the same
-    code). mass_rtol replaces the 1e-4 mass tolerance where the inputs make fp32 logits too coarse for it."""
+    code). mass_rtol replaces the 1e-4 mass tolerance, and lse_rtol widens the lse tolerance by that fraction of
+    |lse|, where the inputs make fp32 logits too coarse for the defaults."""
     q, k, v = device_inputs(layer)
     buf = LayerBuffers.for_config(cfg)
     scale = scale_of(cfg)
@@ -60,7 +61,11 @@ def _both_ways(cfg, layer, oracle, mass_rtol=None):
     go, valid = item_rows(cfg, items, buf.o.float().cpu().numpy())
     gl, _ = item_rows(cfg, items, buf.lse.cpu().numpy())
     check_output(go[valid], od[valid], f"{cfg.name} dense O")
-    check_lse(gl[valid], ld[valid], f"{cfg.name} dense lse")
+    if lse_rtol:
+        err = np.abs(gl[valid].astype(np.float64) - ld[valid])
+        assert (err <= 1e-3 + lse_rtol * np.abs(ld[valid])).all(), f"{cfg.name} dense lse: max err {err.max():.3e}"
+    else:
+        check_lse(gl[valid], ld[valid], f"{cfg.name} dense lse")
 
 
 @pytest.mark.parametrize("name", ["bf16-3x(5x13x31)-ragged", "bf16-C32-3x(5x13x31)-ragged",
@@ -86,10 +91,12 @@ def test_one_pass_masses_when_the_row_max_grows_far(name, oracle_mod):
     # a middle tile 4x (the reference max moves within the anchor span), the last tile 16x (far past it). The last
     # tile's logits reach about 1000, where one fp32 ulp of the tensor core's accumulation is about 1e-4 of the
     # logit scale times log2(e): both calls then agree with the exact masses to a few 1e-5, at times just above
-    # 1e-4, so this case checks the anchor logic at 5e-4 (a wrong anchor factor would be off by 2^60).
+    # 1e-4, so this case checks the anchor logic at 5e-4 (a wrong anchor factor would be off by 2^60). For the same
+    # reason lse (about 900 here) may be off by more than the usual 1e-3: the worst-case rounding bound of a
+    # 128-term fp32 dot product, 128 * 2^-24 of its magnitude, is added to that tolerance.
     layer = _scale_keys(layer, 512, 768, 2)
     layer = _scale_keys(layer, (n - 1) // 256 * 256, n, 4)
-    _both_ways(cfg, layer, oracle_mod, mass_rtol=5e-4)
+    _both_ways(cfg, layer, oracle_mod, mass_rtol=5e-4, lse_rtol=128 * 2.0 ** -24)
 
 
 def test_one_pass_refusals():
