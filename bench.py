@@ -373,6 +373,7 @@ def run_native(args, cfg):
     t_sparse = max_over_ranks(sum(spa_ms) / 1e3)
     t_prof = max_over_ranks(sum(prof_ms) / 1e3)
     t_sel = max_over_ranks(sum(sel_ms) / 1e3)
+    per_sparse, per_prof, per_sel = t_sparse / args.steps, t_prof / args.steps, t_sel / args.steps
     status = L.losa_get_device_error()
     if status != 0:
         raise RuntimeError(f"device error in timed region: {status}")
@@ -489,14 +490,37 @@ def run_native(args, cfg):
                 "worst_row_recall_mass_rule": round(float(row_tau.min()), 6),
                 "worst_row_recall_topk": round(float(row_topk.min()), 6)}
 
+    # Outside the timed region, after everything that reads this step's masses: the dense step alone (no masses),
+    # which sets construction against one dense step at this shape, and the two-pass profile call (masses from a
+    # second Q K^T pass, no workspace), each timed back to back with CUDA events and its own clock record.
+    if not args.no_extras:
+        def profile_series(reps, **kw):
+            buf.profile(q, k, v, scale, **kw)
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            with ClockSampler(local) as ck:
+                ev[0].record(stream)
+                for _ in range(reps):
+                    buf.profile(q, k, v, scale, **kw)
+                ev[1].record(stream)
+                torch.cuda.synchronize()
+            if L.losa_get_device_error() != 0:
+                raise RuntimeError("device error in the profile series")
+            return ev[0].elapsed_time(ev[1]) / reps, ck.summary()
+
+        t_fwd, ck_fwd = profile_series(3, with_mass=False)
+        t_two, ck_two = profile_series(3, one_pass=False)
+        extras["dense_step_no_mass"] = {"ms": round(t_fwd, 3), "calls": 3, "clocks": ck_fwd,
+                                        "profile_select_over_dense_step": round((per_prof + per_sel) * 1e3 / t_fwd,
+                                                                                3)}
+        extras["dense_profile_two_pass"] = {"ms": round(t_two, 3), "calls": 3, "clocks": ck_two}
+
     pk = peaks()
-    per_sparse = t_sparse / K
-    per_prof = t_prof / K
-    per_sel = t_sel / K
     tr = measured_traffic(cfg.name)
     roof = {
-        "dense_profile": roofline("attn_dense_kernel<1> (losa_dense_profile: dense forward + block masses)", "tensor",
-                                  work["profile_flop"], per_prof, pk, "TFLOP/s", tr.get("dense_profile")),
+        "dense_profile": roofline("attn_dense_kernel<1, 1, 1> (losa_dense_profile_ws: dense forward with the block "
+                                  "masses taken in the same pass)", "tensor", work["profile_flop"], per_prof, pk,
+                                  "TFLOP/s", tr.get("dense_profile")),
         "select": roofline("select_rows + select_hist + select_order + select_scatter (losa_select)", "hbm",
                            work["select_bytes"], per_sel, pk, "GB/s", tr.get("select")),
         # the kept-block target is stated against the bf16 dense peak: the burst GEMM rate is the denominator
@@ -514,6 +538,14 @@ def run_native(args, cfg):
         roof["sparse_attn_tau1"] = roofline("attn_sparse_kernel, every list full (tau = 1)", "tensor",
                                             work_model(cfg, f["nnz_blocks"])["sparse_flop"], f["ms"] / 1e3, pk,
                                             "TFLOP/s", None, peak_kind="burst")
+    if "dense_step_no_mass" in extras:
+        roof["dense_step_no_mass"] = roofline("attn_dense_kernel<0, 1, 0> (losa_dense_profile without masses: the "
+                                              "dense step)", "tensor", work["profile_flop"],
+                                              extras["dense_step_no_mass"]["ms"] / 1e3, pk, "TFLOP/s", None)
+        roof["dense_profile_two_pass"] = roofline("attn_dense_kernel<1, 1, 0> (losa_dense_profile: forward, then a "
+                                                  "second Q K^T pass for the masses)", "tensor",
+                                                  1.5 * work["profile_flop"],
+                                                  extras["dense_profile_two_pass"]["ms"] / 1e3, pk, "TFLOP/s", None)
     dominant = max(("dense_profile", per_prof), ("select", per_sel), ("sparse_attn", per_sparse),
                    key=lambda x: x[1])[0]
     line = {
