@@ -97,6 +97,27 @@ def test_pointer_and_tau_validation(lib):
                              raise_on_error=False) == -1
 
 
+def test_one_pass_profile_host_checks(lib):
+    """losa_dense_profile_ws refuses bad arguments on the host, before it asks the device for its SM count: bad
+    shapes, null or misaligned pointers (the workspace included) and a non-finite scale. The workspace size is 0 for
+    a bad shape and for the fp32 path, which takes no workspace."""
+    for s in (L.make_shape(0, 1000, 1024, 128, 128, 128, "bf16"), L.make_shape(2, 1100, 1024, 128, 128, 128, "bf16"),
+              L.make_shape(2, 1000, 1024, 128, 128, 128, 7), L.make_shape(2, 1000, 1024, 64, 128, 128, "f32")):
+        assert L.losa_dense_profile_workspace_bytes(s) == 0
+    for s in (L.make_shape(0, 1000, 1024, 128, 128, 128, "bf16"), L.make_shape(2, 1100, 1024, 128, 128, 128, "bf16")):
+        assert L.losa_dense_profile_ws(s, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, FAKE, ws_bytes=1 << 30, stream=0,
+                                       raise_on_error=False) == -1
+    s = L.make_shape(2, 1000, 1024, 128, 128, 128, "bf16")
+    for args in ((FAKE + 2, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, FAKE),       # misaligned q
+                 (FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, FAKE + 4),       # misaligned workspace
+                 (FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, 0),              # null workspace
+                 (FAKE, FAKE, FAKE, 0.1, FAKE, 0, FAKE, FAKE),              # masses without lse
+                 (FAKE, FAKE, FAKE, float("nan"), FAKE, FAKE, FAKE, FAKE)):  # non-finite scale
+        assert L.losa_dense_profile_ws(s, *args, ws_bytes=1 << 30, stream=0, raise_on_error=False) == -1
+    with pytest.raises(ValueError):  # a raw workspace pointer needs its size
+        L.losa_dense_profile_ws(s, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, FAKE, FAKE, stream=0)
+
+
 def test_capacity_and_unsupported(lib):
     s = L.make_shape(2, 1000, 1024, 128, 128, 128, "bf16")
     ws = L.losa_select_workspace_bytes(s)
