@@ -83,7 +83,9 @@ losa_status losa_dense_profile(const losa_shape* shape, const void* q, const voi
  * the same arguments and results as losa_dense_profile (same definitions; the masses agree with it and with the exact
  * values within the same 1e-4 relative bound, not bit for bit: the sums run in another order).
  *   workspace : device scratch of at least losa_dense_profile_workspace_bytes(shape) bytes (16-byte aligned),
- *               contents on entry irrelevant; ws_bytes is its size, else LOSA_ERR_CAPACITY before any launch.
+ *               contents on entry irrelevant; ws_bytes is its size, else LOSA_ERR_CAPACITY before any launch
+ *               (LOSA_ERR_CUDA if the current device cannot be queried for its SM count). The scratch is used
+ *               only during the call; concurrent calls need separate workspaces.
  * The forward pass already forms every weight 2^(s c - m c) against the row's running max m; it keeps, per row and
  * key block, the exact sum of those weights (brought to one anchor max per row) in the scratch, and each item's
  * masses are reduced from them once the row's final log-sum-exp is known: one pass over the keys instead of two.
