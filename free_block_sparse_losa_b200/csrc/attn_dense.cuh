@@ -1,4 +1,4 @@
-// Dense-step tensor-core kernel (bf16, head_dim 128, 128-row query blocks): attn_dense_kernel<WITH_MASS, SUB>.
+// Dense-step tensor-core kernel (bf16, head_dim 128, 128-row query blocks): attn_dense_kernel<WITH_MASS, SUB, ONE_PASS>.
 //
 // The dense forward (LoSA page, Motivation Summary: A = softmax(Q K^T / sqrt(d)) and O = A V) and, with WITH_MASS, the
 // exact block masses of the construction step (Motivation Summary: M(i, j) = sum of A over query block i and key
@@ -17,9 +17,12 @@
 //   N = 128 instructions (keys 0..127 and 128..255) with P read from TMEM and V from shared memory (MN-major).
 //   Warp 0 issues the TMA loads of Q (once per item) and K (single-buffered), warp 2 those of V (double-buffered),
 //   64 KB per 256-key tile; each box of a tile comes from its own lane. Warp 1 issues the MMAs and owns TMEM.
-//   Mass phase (same item, Q still in shared memory, lse exact in registers): S is recomputed for every 256-key tile
-//   and each warpgroup sums 2^(s*c - lse2) over its 128 columns per key block; per-warp partials go to the idle V
-//   buffer and are flushed to M every 1024 blocks.
+//   One-pass masses (ONE_PASS): every forward tile's exact per-block sums of its weights, brought to a per-row anchor
+//   max, are stored to a [SMs][nk][128] fp32 workspace; once the item's rows have their final max and sum, eight
+//   warps reduce them to M with one factor per row (passed through shared memory).
+//   Two-pass masses (mass phase: same item, Q still in shared memory, lse exact in registers): S is recomputed for
+//   every 256-key tile and each warpgroup sums 2^(s*c - lse2) over its 128 columns per key block; per-warp partials
+//   go to the idle V buffer and are flushed to M every 1024 blocks.
 // Registers: the producer / MMA warpgroup drops to 56 per thread and the softmax warpgroups rise to 224 (setmaxnreg), so
 // the softmax's 128 S values, 64 P words and sums stay in registers.
 // Every wait is bounded in time (LOSA_ERR_TIMEOUT in the device error word, then a clean exit).
